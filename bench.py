@@ -1,0 +1,396 @@
+"""Benchmark: prefill unmasked TFLOP/s (and decode HBM GB/s) of the attention
+core on B200, as a fraction of the measured peaks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--no-decode]
+
+One step = one swa_attn_prefill call (RoPE of the keys, then the fused
+tcgen05 attention kernel with RoPE on the Q tile load, banded causal mask,
+online softmax, P.V and the head gate) over one batch of the Step-3.7-Flash
+sliding-layer workload (B1 S8192 Hq96 Hkv8 W512, theta 1e4).  Inputs are
+resident in HBM and rotate over 4 copies of 439 MB each (more than the
+126 MB L2), so no step reads the previous step's data from L2.
+
+With torchrun (N > 1) every rank runs the same workload on its own GPU (the
+work shards by sequence / kv-head with no exchange; weak scaling); time is
+the max over ranks of the device-timed region.
+
+--impl reference times the CPU oracle (the plain fp64 definition, OpenMP over
+rows) on a bounded row sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from full_gqa_attention_swa_b200 import configs, inputs  # noqa: E402
+
+METRIC = "prefill unmasked TFLOP/s & decode HBM GB/s, as fraction of B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+N_ROTATE = 4
+
+
+# --------------------------------------------------------------- arithmetic
+
+def visible_pairs(S: int, window: int) -> int:
+    """Number of (i, j) with j visible to i: i-W < j <= i (W<0: j <= i)."""
+    if window < 0 or window >= S:
+        return S * (S + 1) // 2
+    W = window
+    return W * (W + 1) // 2 + (S - W) * W
+
+
+def prefill_flops(c) -> float:
+    """Unmasked FLOPs: QK^T and P.V over visible pairs, 2 * 2 * D each."""
+    return 4.0 * 128 * c.Hq * c.B * visible_pairs(c.S, c.window)
+
+
+def prefill_bytes(c) -> int:
+    """Algorithmic HBM bytes: read Q, K, V, gate; write out."""
+    q = c.B * c.S * c.Hq * 128 * 2
+    kv = 2 * c.B * c.S * c.Hkv * 128 * 2
+    gate = c.B * c.S * c.Hq * 4
+    return 2 * q + kv + gate
+
+
+def decode_bytes(c, lens) -> int:
+    """Cache bytes read once per kv-head (K and V) plus q, gate and out."""
+    W = c.window
+    keys = sum(min(int(L), W) if W > 0 else int(L) for L in lens)
+    return keys * c.Hkv * 128 * 2 * 2 + c.B * c.Hq * (128 * 2 * 2 + 4)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def combine_ranks(elapsed_ms_per_rank, n_gpus: int, units_per_rank: float):
+    """Whole-job throughput: units of all ranks over the slowest rank's time."""
+    t = max(elapsed_ms_per_rank)
+    return n_gpus * units_per_rank / (t / 1e3), t
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no samples
+            self.nv = None
+
+    def _sample(self):
+        mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        try:
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append(mhz)
+        for bit, name in self.REASONS.items():
+            if r & bit and bit != 0x1:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.nv:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- GPU legs
+
+def _layer(c):
+    from full_gqa_attention_swa_b200 import api
+
+    return api.LayerParams(c.Hq, c.Hkv, 128, c.window, c.theta, c.rotary_dim)
+
+
+def bench_prefill(c, steps: int, warmup: int, dev, dist=None):
+    from full_gqa_attention_swa_b200 import api
+
+    p = _layer(c)
+    sets = [inputs.prefill_inputs(c.B, c.S, c.Hq, c.Hkv, 128, c.seed + 17 * r, device=dev)
+            for r in range(N_ROTATE)]
+    out = torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws_bytes = api.prefill_workspace_size(p, c.B, c.S)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        d = sets[i % N_ROTATE]
+        api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"], out=out, workspace=ws, stream=stream)
+
+    for i in range(max(warmup, 0)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for i in range(steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    launches = steps * (2 if ws_bytes > 0 else 1)
+    return ms, clocks.summary(), launches
+
+
+def bench_prefill_e2e(c, steps: int, dev):
+    """Same metric through the public API with host buffers: pinned host
+    inputs copied in and the output copied back every step."""
+    from full_gqa_attention_swa_b200 import api
+
+    p = _layer(c)
+    host = inputs.prefill_inputs(c.B, c.S, c.Hq, c.Hkv, 128, c.seed)
+    host = {k: t.pin_memory() for k, t in host.items()}
+    out_host = torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16).pin_memory()
+    d = {k: torch.empty_like(t, device=dev) for k, t in host.items()}
+    out = torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(api.prefill_workspace_size(p, c.B, c.S), 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for k in d:
+            d[k].copy_(host[k], non_blocking=True)
+        api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"], out=out, workspace=ws, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    return ev0.elapsed_time(ev1), h2d, d2h
+
+
+def bench_decode(c, steps: int, warmup: int, dev):
+    from full_gqa_attention_swa_b200 import api
+
+    p = _layer(c)
+    lens = inputs.uniform_int(c.B, c.len_lo, c.len_hi, c.seed)
+    # full layers: caches far larger than L2, one copy; sliding rings (134 MB,
+    # about L2-sized): rotate 4 copies
+    n_sets = 1 if c.window < 0 else N_ROTATE
+    sets = [inputs.decode_inputs(c.B, c.Hq, c.Hkv, 128, c.capacity, c.seed + r, device=dev) for r in range(n_sets)]
+    lens_d = lens.to(dev)
+    max_len = int(lens.max())
+    out = torch.empty(c.B, c.Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(api.decode_workspace_size(p, c.B, max_len), 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        d = sets[i % n_sets]
+        api.attn_decode(p, d["q"], d["gate"], d["k_cache"], d["v_cache"], lens_d, max_len, out=out, workspace=ws,
+                        stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / steps
+    nbytes = decode_bytes(c, lens.tolist())
+    del sets
+    torch.cuda.empty_cache()
+    return ms, nbytes
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_sample_rate(c, budget_s: float, threads: int = 0):
+    """Time the oracle on a growing seeded row sample of the workload until
+    about budget_s seconds; returns (TFLOP/s, rows, seconds, threads)."""
+    import oracle
+
+    lay = oracle.Layer(c.Hq, c.Hkv, 128, c.window, c.theta, c.rotary_dim)
+    d = inputs.prefill_inputs(c.B, c.S, c.Hq, c.Hkv, 128, c.seed)
+    qb, kb, vb = (inputs.as_bits(d[k]) for k in ("q", "k", "v"))
+    g = d["gate"].numpy()
+    rng = np.random.default_rng(c.seed)
+    n = 64
+    while True:
+        rows = np.stack([rng.integers(0, c.B, n), rng.integers(0, c.S, n), rng.integers(0, c.Hq, n)], 1)
+        t0 = time.perf_counter()
+        oracle.prefill(lay, qb, kb, vb, g, rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n >= 1 << 20:
+            break
+        n = int(n * min(8.0, max(2.0, budget_s / max(dt, 1e-3))))
+    W = c.window
+    pairs = sum(min(int(i) + 1, W) if W > 0 else int(i) + 1 for i in rows[:, 1])
+    flops = 4.0 * 128 * pairs
+    return flops / dt / 1e12, n, dt, (threads or oracle.num_threads())
+
+
+# --------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default=configs.STEP_SLIDING.name, choices=sorted(configs.PREFILL))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    c = configs.PREFILL[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    flops = prefill_flops(c)
+    cfg = {"workload": c.name, "global_batch": c.B * world, "seq_len": c.S, "q_heads": c.Hq, "kv_heads": c.Hkv,
+           "head_dim": 128, "window": c.window, "rope_theta": c.theta, "rotary_dim": c.rotary_dim,
+           "parallelism": f"replicas{world}" if world > 1 else "single",
+           "l2": f"rotating {N_ROTATE} input sets of {prefill_bytes(c) / 1e6:.0f} MB (> 126 MB L2)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        rates = []
+        for _ in range(max(args.warmup, 0)):
+            oracle_sample_rate(c, 0.5)
+        t_all = 0.0
+        for _ in range(max(args.steps, 1)):
+            r, n, dt, thr = oracle_sample_rate(c, min(2.0, 60.0 / max(args.steps, 1)))
+            rates.append(r)
+            t_all += dt
+        v = float(np.mean(rates))
+        sample = f"seeded random (b, i, h) rows of {c.name}, ~{n} rows per step"
+        line = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * t_all / max(args.steps, 1), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+                "impl": "reference",
+                "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": sample},
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    from full_gqa_attention_swa_b200 import api
+
+    api.load()
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+
+    ms, clocks, launches = bench_prefill(c, args.steps, max(args.warmup, 3), dev, dist)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value, _ = combine_ranks([ms], world, flops * args.steps / 1e12)   # TFLOP/s over all ranks
+    per_step_ms = ms / args.steps
+    achieved = flops / (per_step_ms / 1e3) / 1e12
+    assert api.device_error() == 0, "a kernel reported a bounded-wait timeout"
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": per_step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic N(0,1) bf16 q/k/v, N(0,1) fp32 gate logits (seeded)", "config": cfg,
+            "clocks": clocks, "gpu_launches": launches}
+    line["roofline"] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                        "peak_source": f"{peak_src} bf16 burst",
+                        "kernel": "swa_attn_prefill (key-RoPE pre-pass + attention kernel), CUDA events"}
+    if rank == 0:
+        e2e_steps = max(3, min(args.steps, 30))
+        e_ms, h2d, d2h = bench_prefill_e2e(c, e2e_steps, dev)
+        line["e2e"] = {"value": flops * e2e_steps / (e_ms / 1e3) / 1e12 * world, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        if not args.no_decode:
+            extra = {}
+            for dc in (configs.DECODE_SLIDING, configs.DECODE_FULL):
+                steps = 200 if dc.window > 0 else 10
+                d_ms, nbytes = bench_decode(dc, steps, 3, dev)
+                gbs = nbytes / (d_ms / 1e3) / 1e9
+                extra[dc.name] = {"ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                                  "peak_source": f"{peak_src} hbm copy"}
+            line["decode"] = extra
+        r, n, dt, thr = oracle_sample_rate(c, args.cpu_budget)
+        line["cpu_baseline"] = {"value": r, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                "sample": f"{n} seeded random (b, i, h) rows of {c.name}, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

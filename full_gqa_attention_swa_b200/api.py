@@ -1,0 +1,227 @@
+"""ctypes binding of libswa.so (include/swa.h), same names as the C ABI.
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+kernels behind the C ABI.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if libswa.so is missing or a call fails, this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libswa.so")
+
+WINDOW_FULL = -1
+
+SWA_OK = 0
+STATUS_NAMES = {0: "SWA_OK", 1: "SWA_ERR_INVALID_ARG", 2: "SWA_ERR_UNSUPPORTED", 3: "SWA_ERR_WORKSPACE",
+                4: "SWA_ERR_CUDA"}
+
+# every function include/swa.h declares
+SYMBOLS = ("swa_rope_qk", "swa_prefill_workspace_size", "swa_attn_prefill", "swa_decode_workspace_size",
+           "swa_attn_decode", "swa_kv_cache_bytes", "swa_status_string", "swa_last_error_detail",
+           "swa_device_error", "swa_version")
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("rope_theta", ctypes.c_double),
+        ("rotary_dim", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+    ]
+
+
+@dataclass(frozen=True)
+class LayerParams:
+    """swa_layer_params: window -1 = full causal; rope_theta 0 = no RoPE;
+    softmax_scale <= 0 = 1/sqrt(head_dim)."""
+
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int = 128
+    window: int = WINDOW_FULL
+    rope_theta: float = 10000.0
+    rotary_dim: int = 128
+    softmax_scale: float = 0.0
+
+    def c(self) -> _Params:
+        return _Params(self.num_q_heads, self.num_kv_heads, self.head_dim, self.window, float(self.rope_theta),
+                       self.rotary_dim, float(self.softmax_scale))
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libswa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m full_gqa_attention_swa_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(_Params)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.swa_rope_qk.argtypes = [P, i32, i32, vp, vp, vp, i32, vp, vp, vp, i32, vp]
+    lib.swa_rope_qk.restype = ctypes.c_int
+    lib.swa_prefill_workspace_size.argtypes = [P, i32, i32]
+    lib.swa_prefill_workspace_size.restype = sz
+    lib.swa_attn_prefill.argtypes = [P, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.swa_attn_prefill.restype = ctypes.c_int
+    lib.swa_decode_workspace_size.argtypes = [P, i32, i32]
+    lib.swa_decode_workspace_size.restype = sz
+    lib.swa_attn_decode.argtypes = [P, i32, vp, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]
+    lib.swa_attn_decode.restype = ctypes.c_int
+    lib.swa_kv_cache_bytes.argtypes = [P, i64, i64]
+    lib.swa_kv_cache_bytes.restype = i64
+    lib.swa_status_string.argtypes = [ctypes.c_int]
+    lib.swa_status_string.restype = ctypes.c_char_p
+    lib.swa_last_error_detail.argtypes = []
+    lib.swa_last_error_detail.restype = ctypes.c_char_p
+    lib.swa_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), i32]
+    lib.swa_device_error.restype = ctypes.c_int
+    lib.swa_version.argtypes = []
+    lib.swa_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != SWA_OK:
+        detail = load().swa_last_error_detail().decode()
+        raise SwaError(status, detail)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def version() -> str:
+    return load().swa_version().decode()
+
+
+def kv_cache_bytes(layer: LayerParams, batch: int, context: int) -> int:
+    return int(load().swa_kv_cache_bytes(ctypes.byref(layer.c()), batch, context))
+
+
+def rope_qk(layer: LayerParams, q=None, k=None, pos=None, pos0: int = 0, v=None, k_cache=None, v_cache=None,
+            stream=None):
+    """swa_rope_qk: rotate q [B,S,Hq,D] / k [B,S,Hkv,D] in place at pos [B,S]
+    (int32) or pos0 + s; optionally append rotated k and v to the cache
+    [B,Hkv,C,D]."""
+    ref = q if q is not None else k
+    if ref is None:
+        return
+    B, S = ref.shape[0], ref.shape[1]
+    D = layer.head_dim
+    _need(q, "q", torch.bfloat16, None if q is None else (B, S, layer.num_q_heads, D))
+    _need(k, "k", torch.bfloat16, None if k is None else (B, S, layer.num_kv_heads, D))
+    _need(v, "v", torch.bfloat16, None if v is None else (B, S, layer.num_kv_heads, D))
+    _need(pos, "pos", torch.int32, None if pos is None else (B, S))
+    C = 0
+    if k_cache is not None:
+        C = k_cache.shape[2]
+        _need(k_cache, "k_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+        _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _check(load().swa_rope_qk(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(pos), int(pos0), _ptr(v),
+                              _ptr(k_cache), _ptr(v_cache), C, _stream(stream)))
+
+
+def prefill_workspace_size(layer: LayerParams, B: int, S: int) -> int:
+    return int(load().swa_prefill_workspace_size(ctypes.byref(layer.c()), B, S))
+
+
+def attn_prefill(layer: LayerParams, q, k, v, gate=None, out=None, workspace=None, stream=None):
+    """swa_attn_prefill on un-rotated q [B,S,Hq,D], k/v [B,S,Hkv,D] (bf16);
+    gate [B,S,Hq] fp32 or None.  Returns out [B,S,Hq,D] bf16."""
+    B, S = q.shape[0], q.shape[1]
+    D = layer.head_dim
+    _need(q, "q", torch.bfloat16, (B, S, layer.num_q_heads, D))
+    _need(k, "k", torch.bfloat16, (B, S, layer.num_kv_heads, D))
+    _need(v, "v", torch.bfloat16, (B, S, layer.num_kv_heads, D))
+    _need(gate, "gate", torch.float32, (B, S, layer.num_q_heads))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, (B, S, layer.num_q_heads, D))
+    need = prefill_workspace_size(layer, B, S)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().swa_attn_prefill(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(v), _ptr(gate),
+                                   _ptr(out), _ptr(workspace), nbytes, _stream(stream)))
+    return out
+
+
+def decode_workspace_size(layer: LayerParams, B: int, max_len: int) -> int:
+    return int(load().swa_decode_workspace_size(ctypes.byref(layer.c()), B, max_len))
+
+
+def attn_decode(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens, max_len: int, out=None, workspace=None,
+                stream=None):
+    """swa_attn_decode: q [B,Hq,D] (rotated), gate [B,Hq] fp32 or None, caches
+    [B,Hkv,C,D], seq_lens [B] int32 (device, counts the current token).
+    Returns out [B,Hq,D] bf16."""
+    B = q.shape[0]
+    D = layer.head_dim
+    C = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (B, layer.num_q_heads, D))
+    _need(gate, "gate", torch.float32, (B, layer.num_q_heads))
+    _need(k_cache, "k_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, (B, layer.num_q_heads, D))
+    need = decode_workspace_size(layer, B, max_len)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().swa_attn_decode(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache), _ptr(v_cache), C,
+                                  _ptr(seq_lens), int(max_len), _ptr(out), _ptr(workspace), nbytes,
+                                  _stream(stream)))
+    return out
+
+
+def device_error(reset: bool = True) -> int:
+    """swa_device_error: synchronise and read (optionally clear) the device
+    error word; 0 means no kernel gave up on a wait."""
+    code = ctypes.c_int32(0)
+    _check(load().swa_device_error(ctypes.byref(code), 1 if reset else 0))
+    return int(code.value)

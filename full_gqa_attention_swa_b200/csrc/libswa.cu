@@ -1,0 +1,364 @@
+// libswa.so: the C ABI declared in include/swa.h.  This file validates
+// arguments, plans workspaces and launch shapes, encodes the TMA tensor maps,
+// and launches the kernels on the caller's stream.  It is built as a single
+// translation unit together with the kernel headers it includes.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/swa.h"
+#include "swa_internal.cuh"
+
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "rope.cuh"
+
+namespace {
+
+using swa::kHeadDim;
+
+thread_local char g_detail[512] = "";
+
+swa_status fail(swa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+swa_status ok() {
+  g_detail[0] = '\0';
+  return SWA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+swa_status check_layer(const swa_layer_params* p) {
+  if (!p) return fail(SWA_ERR_INVALID_ARG, "params is NULL");
+  if (p->num_q_heads < 1 || p->num_kv_heads < 1)
+    return fail(SWA_ERR_INVALID_ARG, "head counts must be >= 1 (Hq=%d, Hkv=%d)", p->num_q_heads, p->num_kv_heads);
+  if (p->num_q_heads % p->num_kv_heads != 0)
+    return fail(SWA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", p->num_q_heads, p->num_kv_heads);
+  if (p->head_dim <= 0) return fail(SWA_ERR_INVALID_ARG, "head_dim must be positive");
+  if (p->head_dim != kHeadDim) return fail(SWA_ERR_UNSUPPORTED, "head_dim=%d (only 128 is supported)", p->head_dim);
+  if (p->window == 0 || p->window < -1)
+    return fail(SWA_ERR_INVALID_ARG, "window=%d (>= 1, or SWA_WINDOW_FULL)", p->window);
+  if (!(p->rope_theta >= 0.0) || !isfinite(p->rope_theta))
+    return fail(SWA_ERR_INVALID_ARG, "rope_theta must be finite and >= 0");
+  if (p->rotary_dim < 0 || p->rotary_dim > p->head_dim || (p->rotary_dim & 1))
+    return fail(SWA_ERR_INVALID_ARG, "rotary_dim=%d (even, 0..head_dim)", p->rotary_dim);
+  if (!isfinite(p->softmax_scale)) return fail(SWA_ERR_INVALID_ARG, "softmax_scale is not finite");
+  return SWA_OK;
+}
+
+bool rotates(const swa_layer_params* p) { return p->rope_theta > 0.0 && p->rotary_dim > 0; }
+
+float scale_log2(const swa_layer_params* p) {
+  const double s = p->softmax_scale > 0.f ? (double)p->softmax_scale : 1.0 / sqrt((double)p->head_dim);
+  return (float)(s * 1.4426950408889634);  // log2(e)
+}
+
+void fill_inv_freq(const swa_layer_params* p, double* inv_freq) {
+  for (int k = 0; k < swa::kMaxRotaryHalf; ++k) inv_freq[k] = 0.0;
+  if (!rotates(p)) return;
+  for (int k = 0; k < p->rotary_dim / 2; ++k)
+    inv_freq[k] = pow(p->rope_theta, -2.0 * (double)k / (double)p->rotary_dim);
+}
+
+// ------------------------------------------------------------ TMA encoding
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map of rank 3 or 4 with a 128-byte swizzled box whose inner
+// extent is 64 elements.  dims/strides as in cuTensorMapEncodeTiled (strides
+// in bytes for dims 1..rank-1).
+swa_status encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return SWA_OK;
+}
+
+// [B, S, H, D] bf16 -> 4-D map {D, H, S, B}, box {64, 1, rows, 1}.
+swa_status encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int rows) {
+  const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)H * kHeadDim * 2,
+                                 (cuuint64_t)S * H * kHeadDim * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  return encode_bf16(map, base, 4, dims, strides, box);
+}
+
+// [B*Hkv, C, D] bf16 cache -> 3-D map {D, C, B*Hkv}, box {64, rows, 1}.
+swa_status encode_cache(CUtensorMap* map, const void* base, int BH, int C, int rows) {
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)C, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)C * kHeadDim * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  return encode_bf16(map, base, 3, dims, strides, box);
+}
+
+swa_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SWA_OK;
+  return fail(SWA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------ planning
+
+struct PrefillPlan {
+  bool rotate;
+  size_t k_bytes, table_bytes, total;
+};
+
+PrefillPlan plan_prefill(const swa_layer_params* p, int B, int S) {
+  PrefillPlan pl{};
+  pl.rotate = rotates(p);
+  if (pl.rotate) {
+    pl.k_bytes = round_up((size_t)B * S * p->num_kv_heads * kHeadDim * 2, 256);
+    pl.table_bytes = round_up((size_t)S * (p->rotary_dim / 2) * sizeof(float2), 256);
+  }
+  pl.total = pl.k_bytes + pl.table_bytes;
+  return pl;
+}
+
+struct DecodePlan {
+  int chunk, splits;
+  size_t o_bytes, ml_bytes, total;
+};
+
+DecodePlan plan_decode(const swa_layer_params* p, int B, int max_len) {
+  DecodePlan pl{};
+  const long long kb = swa::kDecodeKeyBlock;
+  const long long n_vis = p->window > 0 ? (max_len < p->window ? max_len : p->window) : max_len;
+  // aim for about three resident CTAs per SM over the whole batch
+  long long c = ((long long)B * p->num_kv_heads * n_vis + 148 * 3 - 1) / (148 * 3);
+  c = (c + kb - 1) / kb * kb;
+  if (c < 256) c = 256;
+  if (c > 4096) c = 4096;
+  if (c >= n_vis) {
+    pl.chunk = (int)((n_vis + kb - 1) / kb * kb);
+    pl.splits = 1;
+  } else {
+    pl.chunk = (int)c;
+    pl.splits = (int)((n_vis + c - 1) / c);
+  }
+  if (pl.splits > 1) {
+    const size_t rows = (size_t)B * p->num_q_heads * pl.splits;
+    pl.o_bytes = round_up(rows * kHeadDim * sizeof(float), 256);
+    pl.ml_bytes = round_up(rows * sizeof(float2), 256);
+  }
+  pl.total = pl.o_bytes + pl.ml_bytes;
+  return pl;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* swa_version(void) { return "swa-b200 0.1 (sm_100a)"; }
+
+const char* swa_status_string(swa_status s) {
+  switch (s) {
+    case SWA_OK: return "SWA_OK";
+    case SWA_ERR_INVALID_ARG: return "SWA_ERR_INVALID_ARG";
+    case SWA_ERR_UNSUPPORTED: return "SWA_ERR_UNSUPPORTED";
+    case SWA_ERR_WORKSPACE: return "SWA_ERR_WORKSPACE";
+    case SWA_ERR_CUDA: return "SWA_ERR_CUDA";
+  }
+  return "SWA_ERR_UNKNOWN";
+}
+
+const char* swa_last_error_detail(void) { return g_detail; }
+
+swa_status swa_device_error(int32_t* code, int32_t reset) {
+  if (!code) return fail(SWA_ERR_INVALID_ARG, "code is NULL");
+  swa_status st = cuda_status(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+  if (st != SWA_OK) return st;
+  int v = 0;
+  st = cuda_status(cudaMemcpyFromSymbol(&v, swa::g_device_error, sizeof(int)), "read device error word");
+  if (st != SWA_OK) return st;
+  *code = v;
+  if (reset) {
+    const int zero = 0;
+    st = cuda_status(cudaMemcpyToSymbol(swa::g_device_error, &zero, sizeof(int)), "reset device error word");
+    if (st != SWA_OK) return st;
+  }
+  return ok();
+}
+
+int64_t swa_kv_cache_bytes(const swa_layer_params* p, int64_t batch, int64_t context) {
+  if (check_layer(p) != SWA_OK || batch < 0 || context < 0) return -1;
+  const int64_t C = (p->window > 0 && context > p->window) ? p->window : context;
+  return batch * p->num_kv_heads * C * p->head_dim * 2 * 2;
+}
+
+swa_status swa_rope_qk(const swa_layer_params* p, int32_t B, int32_t S, uint16_t* q, uint16_t* k,
+                       const int32_t* pos, int32_t pos0, const uint16_t* v, uint16_t* k_cache, uint16_t* v_cache,
+                       int32_t cache_capacity, void* stream) {
+  swa_status st = check_layer(p);
+  if (st != SWA_OK) return st;
+  if (B < 0 || S < 0) return fail(SWA_ERR_INVALID_ARG, "B=%d S=%d must be >= 0", B, S);
+  const bool cache = k_cache || v_cache;
+  if (cache && !(k_cache && v_cache)) return fail(SWA_ERR_INVALID_ARG, "k_cache and v_cache must both be given");
+  if (cache && (!k || !v)) return fail(SWA_ERR_INVALID_ARG, "the cache append needs k and v");
+  if (cache) {
+    if (cache_capacity < 1) return fail(SWA_ERR_INVALID_ARG, "cache_capacity=%d", cache_capacity);
+    if (p->window > 0 && cache_capacity != p->window)
+      return fail(SWA_ERR_INVALID_ARG, "sliding layer: cache_capacity=%d must equal window=%d", cache_capacity,
+                  p->window);
+  }
+  if (!pos && pos0 < 0) return fail(SWA_ERR_INVALID_ARG, "pos0=%d must be >= 0", pos0);
+  const void* ptrs[] = {q, k, v, k_cache, v_cache, pos};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(SWA_ERR_INVALID_ARG, "tensor pointer %p is not 16-byte aligned", ptr);
+  if ((long long)B * S == 0 || (!q && !k)) return ok();
+  if ((long long)B * S * 16 / 256 > 0x7FFFFFFFll) return fail(SWA_ERR_UNSUPPORTED, "too many tokens");
+  swa::RopeArgs a{};
+  a.B = B; a.S = S; a.Hq = p->num_q_heads; a.Hkv = p->num_kv_heads;
+  a.rotary_dim = p->rotary_dim; a.pos0 = pos0; a.pos = pos;
+  a.rotate = rotates(p) ? 1 : 0;
+  a.q = q; a.k_src = k; a.k_dst = k; a.v = v;
+  a.k_cache = k_cache; a.v_cache = v_cache; a.cache_capacity = cache_capacity; a.window = p->window;
+  a.table = nullptr;
+  fill_inv_freq(p, a.inv_freq);
+  if (!a.rotate && !cache) return ok();
+  st = cuda_status(swa::launch_rope(a, (cudaStream_t)stream), "rope launch");
+  return st == SWA_OK ? ok() : st;
+}
+
+size_t swa_prefill_workspace_size(const swa_layer_params* p, int32_t B, int32_t S) {
+  if (check_layer(p) != SWA_OK || B < 0 || S < 0) return 0;
+  return plan_prefill(p, B, S).total;
+}
+
+swa_status swa_attn_prefill(const swa_layer_params* p, int32_t B, int32_t S, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const float* gate, uint16_t* out, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  swa_status st = check_layer(p);
+  if (st != SWA_OK) return st;
+  if (B < 0 || S < 0) return fail(SWA_ERR_INVALID_ARG, "B=%d S=%d must be >= 0", B, S);
+  if ((long long)B * S == 0) return ok();
+  if (!q || !k || !v || !out) return fail(SWA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  const void* ptrs[] = {q, k, v, out, gate, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(SWA_ERR_INVALID_ARG, "tensor pointer %p is not 16-byte aligned", ptr);
+  const PrefillPlan pl = plan_prefill(p, B, S);
+  if (pl.total > 0) {
+    if (!workspace) return fail(SWA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", pl.total);
+    if (workspace_bytes < pl.total)
+      return fail(SWA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, pl.total);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(SWA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  const int Hq = p->num_q_heads, Hkv = p->num_kv_heads, G = Hq / Hkv;
+  const long long n_q_tiles = ((long long)S + 127) / 128;
+  const long long n_cta = n_q_tiles * ((G + 1) / 2) * Hkv * (long long)B;
+  if (n_cta > 0x7FFFFFFFll) return fail(SWA_ERR_UNSUPPORTED, "grid too large (%lld tiles)", n_cta);
+
+  cudaStream_t s = (cudaStream_t)stream;
+  const uint16_t* k_att = k;
+  float2* table = nullptr;
+  if (pl.rotate) {
+    uint16_t* k_rot = reinterpret_cast<uint16_t*>(workspace);
+    table = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace) + pl.k_bytes);
+    swa::RopeArgs r{};
+    r.B = B; r.S = S; r.Hq = Hq; r.Hkv = Hkv; r.rotary_dim = p->rotary_dim; r.pos0 = 0; r.pos = nullptr;
+    r.q = nullptr; r.k_src = k; r.k_dst = k_rot; r.v = nullptr; r.k_cache = nullptr; r.v_cache = nullptr;
+    r.cache_capacity = 0; r.window = p->window; r.table = table; r.rotate = 1;
+    fill_inv_freq(p, r.inv_freq);
+    st = cuda_status(swa::launch_rope(r, s), "rope (keys) launch");
+    if (st != SWA_OK) return st;
+    k_att = k_rot;
+  }
+  CUtensorMap qm, km, vm;
+  if ((st = encode_bshd(&qm, q, B, S, Hq, 128)) != SWA_OK) return st;
+  if ((st = encode_bshd(&km, k_att, B, S, Hkv, 128)) != SWA_OK) return st;
+  if ((st = encode_bshd(&vm, v, B, S, Hkv, 128)) != SWA_OK) return st;
+  swa::PrefillArgs a{};
+  a.B = B; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.window = p->window;
+  a.rotary_dim = pl.rotate ? p->rotary_dim : 0;
+  a.scale_log2 = scale_log2(p);
+  a.table = table;
+  a.gate = gate;
+  a.out = out;
+  a.n_q_tiles = (int)n_q_tiles;
+  a.n_head_pairs = (G + 1) / 2;
+  st = cuda_status(swa::launch_prefill(a, qm, km, vm, s), "prefill launch");
+  return st == SWA_OK ? ok() : st;
+}
+
+size_t swa_decode_workspace_size(const swa_layer_params* p, int32_t B, int32_t max_len) {
+  if (check_layer(p) != SWA_OK || B < 0 || max_len < 1) return 0;
+  return plan_decode(p, B, max_len).total;
+}
+
+swa_status swa_attn_decode(const swa_layer_params* p, int32_t B, const uint16_t* q, const float* gate,
+                           const uint16_t* k_cache, const uint16_t* v_cache, int32_t cache_capacity,
+                           const int32_t* seq_lens, int32_t max_len, uint16_t* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  swa_status st = check_layer(p);
+  if (st != SWA_OK) return st;
+  if (B < 0) return fail(SWA_ERR_INVALID_ARG, "B=%d must be >= 0", B);
+  if (B == 0) return ok();
+  const int Hq = p->num_q_heads, Hkv = p->num_kv_heads, G = Hq / Hkv;
+  if (G > 16) return fail(SWA_ERR_UNSUPPORTED, "decode supports up to 16 q-heads per kv-head (G=%d)", G);
+  if (!q || !k_cache || !v_cache || !seq_lens || !out)
+    return fail(SWA_ERR_INVALID_ARG, "q, k_cache, v_cache, seq_lens and out must be non-NULL");
+  const void* ptrs[] = {q, gate, k_cache, v_cache, seq_lens, out, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(SWA_ERR_INVALID_ARG, "tensor pointer %p is not 16-byte aligned", ptr);
+  if (cache_capacity < 1) return fail(SWA_ERR_INVALID_ARG, "cache_capacity=%d", cache_capacity);
+  if (p->window > 0 && cache_capacity != p->window)
+    return fail(SWA_ERR_INVALID_ARG, "sliding layer: cache_capacity=%d must equal window=%d", cache_capacity,
+                p->window);
+  if (max_len < 1) return fail(SWA_ERR_INVALID_ARG, "max_len=%d must be >= 1", max_len);
+  if (p->window < 0 && max_len > cache_capacity)
+    return fail(SWA_ERR_INVALID_ARG, "full layer: max_len=%d exceeds cache_capacity=%d", max_len, cache_capacity);
+  if ((long long)B * Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B*Hkv=%lld too large", (long long)B * Hkv);
+  const DecodePlan pl = plan_decode(p, B, max_len);
+  if (pl.total > 0) {
+    if (!workspace) return fail(SWA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", pl.total);
+    if (workspace_bytes < pl.total)
+      return fail(SWA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, pl.total);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(SWA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  CUtensorMap km, vm;
+  if ((st = encode_cache(&km, k_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
+  if ((st = encode_cache(&vm, v_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
+  swa::DecodeArgs a{};
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.window = p->window; a.capacity = cache_capacity;
+  a.scale_log2 = scale_log2(p);
+  a.q = q; a.gate = gate; a.seq_lens = seq_lens; a.out = out;
+  a.chunk = pl.chunk; a.max_splits = pl.splits;
+  a.part_o = pl.splits > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
+  a.part_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace) + pl.o_bytes) : nullptr;
+  st = cuda_status(swa::launch_decode(a, km, vm, (cudaStream_t)stream), "decode launch");
+  return st == SWA_OK ? ok() : st;
+}
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+// Rotary position encoding of Q and K (rotate-half pairs over the first
+// rotary_dim dims, angle p * theta^(-2k/rotary_dim)), with an optional append
+// of the rotated key and the raw value into a KV cache (ring slot p mod W on
+// sliding layers, slot p on full layers).
+//
+// Follows the "Step-3.7-Flash-oQ3e" explainer, section 2.3 (per-layer theta,
+// partial rotary on full layers) and section 2.2 (a sliding layer's cache
+// keeps the last W tokens), and the "Muse-Glimmer-30B-6bit" explainer's RoPE
+// section (theta 0 = no rotation).
+//
+// Layout of the work: 16 lanes per (token, head) row, one 16-byte chunk of 8
+// dims per lane.  A lane reads its chunk and, for rotary dims, the partner
+// chunk rotary_dim/2 away, so both halves of a pair are read before any lane
+// of the row writes (a __syncwarp separates reads from writes when rotating in
+// place).  The angle is evaluated in fp64 (p up to 2^31, theta up to 5e6) and
+// its cos/sin rounded to fp32 once per (token, freq); each lane reuses them
+// across all heads it visits.
+#pragma once
+#include "swa_internal.cuh"
+
+namespace swa {
+
+namespace rope_detail {
+
+constexpr int kChunks = kHeadDim / 8;  // 16-byte chunks per head row
+
+struct Chunk {
+  uint4 raw;
+};
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x);
+  f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z);
+  f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(f[0], f[1]);
+  u.y = pack_bf16x2(f[2], f[3]);
+  u.z = pack_bf16x2(f[4], f[5]);
+  u.w = pack_bf16x2(f[6], f[7]);
+  return u;
+}
+
+// Element e (0..7) of this lane's chunk: its rotary role.
+//   role 0: pass-through; role 1: first half (y = x c - x' s);
+//   role 2: second half (y = x c + x' s).  freq index k, partner dim.
+struct LaneRole {
+  int role[8];
+  int freq[8];
+  int partner[8];
+  bool partner_is_chunk;  // partner elements form one aligned chunk
+  int partner_chunk;
+};
+
+__device__ __forceinline__ LaneRole lane_role(int chunk, int r) {
+  LaneRole L;
+  const int half = r / 2;
+  for (int e = 0; e < 8; ++e) {
+    const int d = chunk * 8 + e;
+    if (d < half) {
+      L.role[e] = 1; L.freq[e] = d; L.partner[e] = d + half;
+    } else if (d < r) {
+      L.role[e] = 2; L.freq[e] = d - half; L.partner[e] = d - half;
+    } else {
+      L.role[e] = 0; L.freq[e] = 0; L.partner[e] = d;
+    }
+  }
+  L.partner_is_chunk = (half % 8) == 0 && chunk * 8 < r;
+  L.partner_chunk = chunk * 8 < half ? chunk + half / 8 : chunk - half / 8;
+  return L;
+}
+
+__device__ __forceinline__ void rotate_chunk(const uint16_t* row_src, uint16_t* row_dst, int chunk,
+                                             const LaneRole& L, const float (&c)[8], const float (&s)[8],
+                                             bool active, bool in_place) {
+  uint4 own = make_uint4(0, 0, 0, 0), par = make_uint4(0, 0, 0, 0);
+  float xp[8];
+  if (active) {
+    own = *reinterpret_cast<const uint4*>(row_src + chunk * 8);
+    if (L.partner_is_chunk) {
+      par = *reinterpret_cast<const uint4*>(row_src + L.partner_chunk * 8);
+      unpack8(par, xp);
+    } else {
+      for (int e = 0; e < 8; ++e) {
+        uint32_t b = row_src[L.partner[e]];
+        xp[e] = __uint_as_float(b << 16);
+      }
+    }
+  }
+  if (in_place) __syncwarp();
+  if (active) {
+    float x[8], y[8];
+    unpack8(own, x);
+    for (int e = 0; e < 8; ++e) {
+      if (L.role[e] == 1) y[e] = x[e] * c[e] - xp[e] * s[e];
+      else if (L.role[e] == 2) y[e] = x[e] * c[e] + xp[e] * s[e];
+      else y[e] = x[e];
+    }
+    *reinterpret_cast<uint4*>(row_dst + chunk * 8) = pack8(y);
+  }
+  if (in_place) __syncwarp();
+}
+
+// grid.x: ceil(B*S*16 / blockDim.x); grid.y: head split (heads h with
+// h % gridDim.y == blockIdx.y).
+__global__ void __launch_bounds__(256) rope_kernel(const RopeArgs a) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int chunk = (int)(tid & (kChunks - 1));
+  const long long tok = tid >> 4;
+  const long long n_tok = (long long)a.B * a.S;
+  const bool active = tok < n_tok;
+  const long long tk = active ? tok : 0;
+  const int b = (int)(tk / a.S);
+  const int s_idx = (int)(tk % a.S);
+  const int p = a.pos ? a.pos[tk] : a.pos0 + s_idx;
+
+  const int r = a.rotate ? a.rotary_dim : 0;
+  const LaneRole L = lane_role(chunk, r);
+  float c[8], s[8];
+  for (int e = 0; e < 8; ++e) {
+    if (L.role[e] != 0) {
+      double sd, cd;
+      sincos((double)p * a.inv_freq[L.freq[e]], &sd, &cd);
+      c[e] = (float)cd;
+      s[e] = (float)sd;
+    } else {
+      c[e] = 1.f;
+      s[e] = 0.f;
+    }
+  }
+  if (a.table && active && b == 0 && blockIdx.y == 0) {
+    for (int e = 0; e < 8; ++e)
+      if (L.role[e] == 1) a.table[(long long)s_idx * (r / 2) + L.freq[e]] = make_float2(c[e], s[e]);
+  }
+
+  const int hs = blockIdx.y, nhs = gridDim.y;
+  if (a.q && r > 0) {
+    for (int h = hs; h < a.Hq; h += nhs) {
+      uint16_t* row = a.q + (tk * a.Hq + h) * kHeadDim;
+      rotate_chunk(row, row, chunk, L, c, s, active, true);
+    }
+  }
+  if (a.k_src) {
+    const bool in_place = a.k_dst == a.k_src;
+    long long slot = 0;
+    bool slot_ok = true;
+    if (a.k_cache) {
+      slot = a.window > 0 ? (long long)(p % a.window) : (long long)p;
+      slot_ok = p >= 0 && slot < a.cache_capacity;
+      if (active && !slot_ok && chunk == 0 && hs == 0) record_error(kErrRope + 1);
+    }
+    for (int h = hs; h < a.Hkv; h += nhs) {
+      const uint16_t* src = a.k_src + (tk * a.Hkv + h) * kHeadDim;
+      uint16_t* dst = a.k_dst + (tk * a.Hkv + h) * kHeadDim;
+      if (r > 0 || !in_place) rotate_chunk(src, dst, chunk, L, c, s, active, in_place);
+      if (a.k_cache && active && slot_ok) {
+        // the rotated chunk: re-read from dst when it was written, else rotate here
+        // this lane's own rotated chunk, written above by this same thread
+        const uint4 kv = *reinterpret_cast<const uint4*>(dst + chunk * 8);
+        uint16_t* kc = a.k_cache + (((long long)b * a.Hkv + h) * a.cache_capacity + slot) * kHeadDim;
+        uint16_t* vc = a.v_cache + (((long long)b * a.Hkv + h) * a.cache_capacity + slot) * kHeadDim;
+        *reinterpret_cast<uint4*>(kc + chunk * 8) = kv;
+        *reinterpret_cast<uint4*>(vc + chunk * 8) =
+            *reinterpret_cast<const uint4*>(a.v + (tk * a.Hkv + h) * kHeadDim + chunk * 8);
+      }
+    }
+  }
+}
+
+}  // namespace rope_detail
+
+cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
+  const long long n_tok = (long long)a.B * a.S;
+  if (n_tok == 0) return cudaSuccess;
+  const int threads = 256;
+  const long long lanes = n_tok * rope_detail::kChunks;
+  const long long blocks = (lanes + threads - 1) / threads;
+  // few tokens (decode): spread heads over grid.y so enough warps run
+  int hsplit = 1;
+  const int max_heads = a.Hq > a.Hkv ? a.Hq : a.Hkv;
+  while (blocks * hsplit < 148 * 4 && hsplit < max_heads) hsplit *= 2;
+  if (hsplit > max_heads) hsplit = max_heads;
+  if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  rope_detail::rope_kernel<<<dim3((unsigned)blocks, (unsigned)hsplit), threads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace swa

@@ -1,0 +1,195 @@
+/*
+ * swa.h -- C ABI of libswa.so: the attention core of a hybrid sliding-window /
+ * full-attention GQA decoder layer on NVIDIA B200 (sm_100a).
+ *
+ * The operation (page title, section that defines it):
+ *   - "Step-3.7-Flash-oQ3e" explainer, section 2.2: sliding layers attend
+ *     through a sliding-window causal mask and keep only the last W (= 512)
+ *     tokens of KV cache; full layers use a plain causal mask.  Read here as:
+ *     query i sees key j iff i - W < j <= i (W keys, self included);
+ *     window = SWA_WINDOW_FULL means no lower bound.
+ *   - same page, section 2.3: rope_theta is chosen per layer, partial rotary
+ *     factors rotate only part of each head on full layers, and every head
+ *     has its own sigmoid output gate.  Read here as: the first rotary_dim
+ *     dims are rotated in rotate-half pairs (k, k + rotary_dim/2) by the angle
+ *     p * rope_theta^(-2k/rotary_dim); the gate multiplies the normalised
+ *     attention output of (token, q-head) by sigmoid(gate logit).
+ *   - "Step-3.7-Flash" spec card, config dump: 64 query heads in 8 attention
+ *     groups (att_impl_type GQA).  Read here as: q-head h uses kv-head
+ *     h / (num_q_heads / num_kv_heads).
+ *   - "Muse-Glimmer-30B-6bit" explainer, RoPE section: a layer rope theta of
+ *     0 means the layer applies no rotary encoding.
+ *   Scores are softmax_scale * <q_i, k_j> (default 1/sqrt(head_dim)), the
+ *   masked softmax is taken over the visible keys, and the output is the
+ *   softmax-weighted sum of values.
+ *
+ * Conventions for every call:
+ *   - Tensors are device pointers to contiguous row-major arrays in the layout
+ *     stated at each argument; bf16 tensors are passed as uint16_t (their bit
+ *     patterns).  Every tensor pointer must be 16-byte aligned.
+ *   - The caller owns all memory.  No call allocates device memory; calls that
+ *     need scratch take a caller-provided workspace whose size a *_size()
+ *     query returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and never synchronise the host.
+ *   - Errors: argument problems are reported before anything is launched
+ *     (SWA_ERR_INVALID_ARG / SWA_ERR_UNSUPPORTED / SWA_ERR_WORKSPACE); a
+ *     failed launch returns SWA_ERR_CUDA.  swa_last_error_detail() describes
+ *     the last failure of the calling thread.  Kernels never trap: a device-
+ *     side wait that runs out of time records a code that swa_device_error()
+ *     reads.  No C++ exception crosses this interface.
+ */
+#ifndef SWA_H_
+#define SWA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SWA_API __attribute__((visibility("default")))
+#else
+#define SWA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum swa_status {
+  SWA_OK = 0,
+  SWA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or parameter */
+  SWA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim != 128) */
+  SWA_ERR_WORKSPACE = 3,     /* workspace pointer missing or too small */
+  SWA_ERR_CUDA = 4           /* a CUDA runtime/driver call failed */
+} swa_status;
+
+#define SWA_WINDOW_FULL (-1)
+
+/* One attention layer's parameters. */
+typedef struct swa_layer_params {
+  int32_t num_q_heads;   /* Hq >= 1 */
+  int32_t num_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0 */
+  int32_t head_dim;      /* D; 128 is the only supported value */
+  int32_t window;        /* W >= 1 for a sliding layer; SWA_WINDOW_FULL for full causal */
+  double rope_theta;     /* >= 0; 0 means no rotary encoding */
+  int32_t rotary_dim;    /* even, 0..head_dim; 0 means no rotary encoding */
+  float softmax_scale;   /* > 0, or <= 0 for 1/sqrt(head_dim) */
+} swa_layer_params;
+
+/*
+ * swa_rope_qk -- rotary position encoding of q and k in place, optionally
+ * appending the rotated keys and the raw values to a KV cache.
+ * (Step explainer section 2.3; Muse explainer RoPE section; the cache rule is
+ *  Step explainer section 2.2: a sliding layer keeps the last W tokens.)
+ *
+ *   q        [B, S, Hq, D] bf16, rotated in place; may be NULL.
+ *   k        [B, S, Hkv, D] bf16, rotated in place; may be NULL.
+ *   pos      [B, S] int32 device positions (each >= 0), or NULL: token s of
+ *            every sequence is at position pos0 + s.
+ *   v        [B, S, Hkv, D] bf16; required iff the caches are given.
+ *   k_cache, v_cache  [B, Hkv, C, D] bf16 with C = cache_capacity, or both
+ *            NULL.  Token at position p goes to slot p mod W on a sliding
+ *            layer (C must equal W) and to slot p on a full layer (p < C is
+ *            the caller's promise; C >= 1).  k must be given with caches.
+ *   The angle is p * theta^(-2k/rotary_dim), evaluated in fp64; the
+ *   rotation itself runs in fp32 and the result is rounded to bf16.
+ *   With theta == 0 or rotary_dim == 0, q/k are left unchanged and the
+ *   caches (if any) still receive k and v.
+ */
+SWA_API swa_status swa_rope_qk(const swa_layer_params* params, int32_t B, int32_t S, uint16_t* q, uint16_t* k,
+                       const int32_t* pos, int32_t pos0, const uint16_t* v, uint16_t* k_cache,
+                       uint16_t* v_cache, int32_t cache_capacity, void* stream);
+
+/*
+ * swa_prefill_workspace_size -- bytes of workspace swa_attn_prefill needs for
+ * (params, B, S): the rotated keys [B, S, Hkv, D] bf16 plus the fp32 cos/sin
+ * table of positions 0..S-1, each 256-byte aligned; 0 when the layer applies
+ * no rotary encoding.  Returns 0 for invalid
+ * parameters.
+ */
+SWA_API size_t swa_prefill_workspace_size(const swa_layer_params* params, int32_t B, int32_t S);
+
+/*
+ * swa_attn_prefill -- causal (W infinite) or banded (W finite) GQA attention
+ * of S tokens at positions 0..S-1, RoPE included, with the per-head gate.
+ * (Step explainer sections 2.2 and 2.3; spec card GQA groups.)
+ *
+ *   q      [B, S, Hq, D]  bf16, NOT rotated (RoPE is applied on the tile load)
+ *   k      [B, S, Hkv, D] bf16, NOT rotated
+ *   v      [B, S, Hkv, D] bf16
+ *   gate   [B, S, Hq] fp32 logits, or NULL for no gate
+ *   out    [B, S, Hq, D]  bf16: sigmoid(gate) * softmax(scale q k^T) v,
+ *          accumulated in fp32 and rounded to nearest-even bf16
+ *   workspace / workspace_bytes: at least swa_prefill_workspace_size()
+ *          bytes of device memory, 256-byte aligned; overwritten.
+ *   q, k, v, gate and workspace must not overlap out.
+ */
+SWA_API swa_status swa_attn_prefill(const swa_layer_params* params, int32_t B, int32_t S, const uint16_t* q,
+                            const uint16_t* k, const uint16_t* v, const float* gate, uint16_t* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * swa_decode_workspace_size -- bytes of workspace swa_attn_decode needs for a
+ * batch of B sequences whose lengths are at most max_len (split-K partial
+ * results).  Returns 0 when no workspace is needed or parameters are invalid.
+ */
+SWA_API size_t swa_decode_workspace_size(const swa_layer_params* params, int32_t B, int32_t max_len);
+
+/*
+ * swa_attn_decode -- one query token per sequence against its KV cache.
+ * (Step explainer section 2.2: a sliding layer's cache holds only the last W
+ *  tokens; full layers see the whole history.)
+ *
+ *   q        [B, Hq, D] bf16, ALREADY rotated (swa_rope_qk at p = L_b - 1)
+ *   gate     [B, Hq] fp32 logits, or NULL
+ *   k_cache  [B, Hkv, C, D] bf16 rotated keys; v_cache same shape, raw values
+ *   cache_capacity  C: must equal W on a sliding layer (ring of W slots,
+ *            position p in slot p mod W); on a full layer slot p holds
+ *            position p and C >= every seq_lens[b].
+ *   seq_lens [B] int32 device, 1 <= L_b, counting the current token (already
+ *            appended); the query sits at position L_b - 1 and sees the
+ *            min(L_b, W) filled ring slots (sliding) or slots 0..L_b-1 (full).
+ *   max_len  host-side upper bound of seq_lens (sizes the split grid).
+ *   out      [B, Hq, D] bf16
+ *   workspace / workspace_bytes: at least swa_decode_workspace_size() bytes
+ *            (may be NULL when that is 0); overwritten.
+ *   Cache slots that are not visible are never read as values: they may
+ *   hold anything, including NaN.
+ */
+SWA_API swa_status swa_attn_decode(const swa_layer_params* params, int32_t B, const uint16_t* q, const float* gate,
+                           const uint16_t* k_cache, const uint16_t* v_cache, int32_t cache_capacity,
+                           const int32_t* seq_lens, int32_t max_len, uint16_t* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * swa_kv_cache_bytes -- bytes of one layer's K and V cache for `batch`
+ * sequences of up to `context` tokens: batch x Hkv x C x D x 2 (K and V) x 2
+ * (bf16), with C = min(context, W) on a sliding layer and C = context on a
+ * full layer.  (Muse explainer, GQA section: the per-model footprint is this
+ * summed over layers.)  Returns -1 for invalid arguments.
+ */
+SWA_API int64_t swa_kv_cache_bytes(const swa_layer_params* params, int64_t batch, int64_t context);
+
+/* Human-readable name of a status code (static string). */
+SWA_API const char* swa_status_string(swa_status status);
+
+/* Detail of the calling thread's last failed call (static per-thread buffer;
+ * "" if none). */
+SWA_API const char* swa_last_error_detail(void);
+
+/*
+ * swa_device_error -- reads the device-side error word of the current device
+ * (synchronises the device first).  *code = 0 means no kernel recorded an
+ * error; otherwise the kernel and wait site whose bounded wait ran out
+ * (decimal: kernel * 100 + site).  reset != 0 clears the word afterwards.
+ */
+SWA_API swa_status swa_device_error(int32_t* code, int32_t reset);
+
+/* Library version string. */
+SWA_API const char* swa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H_ */

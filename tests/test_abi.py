@@ -1,0 +1,138 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and
+loads, exports every function include/swa.h declares, sizes workspaces and
+KV caches, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from full_gqa_attention_swa_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "swa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SWA_API\s+[\w\s\*]+?\b(swa_\w+)\s*\(", text)))
+
+
+def _P(**kw):
+    base = dict(num_q_heads=8, num_kv_heads=2, head_dim=128, window=64, rope_theta=1e4, rotary_dim=128,
+                softmax_scale=0.0)
+    base.update(kw)
+    return ctypes.byref(api._Params(**base))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert len(declared) == len(api.SYMBOLS) == 10
+    assert sorted(api.SYMBOLS) == declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert "sm_100a" in api.version()
+
+
+def test_status_strings(lib):
+    for code, name in api.STATUS_NAMES.items():
+        assert lib.swa_status_string(code).decode() == name
+
+
+def test_kv_cache_bytes_matches_page_arithmetic(lib):
+    # Muse explainer, GQA section: 128K context, 2 KV heads, 52 layers ~ 6.5 GiB
+    full = api.LayerParams(32, 2, 128, api.WINDOW_FULL, 0.0, 128)
+    assert 52 * api.kv_cache_bytes(full, 1, 131072) == 6.5 * 2 ** 30
+    mha = api.LayerParams(32, 32, 128, api.WINDOW_FULL, 0.0, 128)
+    assert 52 * api.kv_cache_bytes(mha, 1, 131072) == 104 * 2 ** 30
+    # a sliding layer's ring keeps W slots however long the context
+    sl = api.LayerParams(32, 2, 128, 2048, 5e5, 128)
+    assert api.kv_cache_bytes(sl, 1, 131072) == 2048 * 2 * 128 * 2 * 2
+    assert api.kv_cache_bytes(sl, 3, 100) == 3 * 100 * 2 * 128 * 2 * 2
+    assert lib.swa_kv_cache_bytes(_P(head_dim=64), 1, 1) == -1
+
+
+def test_workspace_sizes(lib):
+    p = api.LayerParams(96, 8, 128, 512, 1e4, 128)
+    ws = api.prefill_workspace_size(p, 1, 8192)
+    k_bytes = 8192 * 8 * 128 * 2
+    table = 8192 * 64 * 8
+    assert ws == k_bytes + table
+    assert api.prefill_workspace_size(api.LayerParams(32, 2, 128, -1, 0.0, 128), 4, 16384) == 0
+    # sliding decode: one split, no workspace; full decode: split-K partials
+    assert api.decode_workspace_size(p, 64, 131072) == 0
+    full = api.LayerParams(64, 8, 128, -1, 5e6, 64)
+    assert api.decode_workspace_size(full, 64, 131072) > 0
+
+
+NULL = None
+FAKE = 1 << 20          # aligned, never dereferenced: every case fails validation first
+MIS = (1 << 20) + 8     # 8-byte aligned only
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_q_heads=8, num_kv_heads=3), 1),
+    (dict(num_kv_heads=0), 1),
+    (dict(head_dim=64), 2),
+    (dict(window=0), 1),
+    (dict(window=-2), 1),
+    (dict(rotary_dim=3), 1),
+    (dict(rotary_dim=130), 1),
+    (dict(rope_theta=-1.0), 1),
+    (dict(rope_theta=float("inf")), 1),
+    (dict(softmax_scale=float("nan")), 1),
+])
+def test_bad_layer_params(lib, kw, status):
+    st = lib.swa_attn_prefill(_P(**kw), 1, 128, FAKE, FAKE, FAKE, NULL, FAKE, FAKE, 1 << 30, NULL)
+    assert st == status
+    assert lib.swa_last_error_detail().decode() != ""
+
+
+def test_prefill_argument_errors(lib):
+    p = _P()
+    assert lib.swa_attn_prefill(None, 1, 128, FAKE, FAKE, FAKE, NULL, FAKE, FAKE, 1 << 30, NULL) == 1
+    assert lib.swa_attn_prefill(p, -1, 128, FAKE, FAKE, FAKE, NULL, FAKE, FAKE, 1 << 30, NULL) == 1
+    assert lib.swa_attn_prefill(p, 1, 128, NULL, FAKE, FAKE, NULL, FAKE, FAKE, 1 << 30, NULL) == 1
+    assert lib.swa_attn_prefill(p, 1, 128, FAKE, FAKE, FAKE, NULL, NULL, FAKE, 1 << 30, NULL) == 1
+    assert lib.swa_attn_prefill(p, 1, 128, MIS, FAKE, FAKE, NULL, FAKE, FAKE, 1 << 30, NULL) == 1
+    assert lib.swa_attn_prefill(p, 1, 128, FAKE, FAKE, FAKE, MIS, FAKE, FAKE, 1 << 30, NULL) == 1
+    assert lib.swa_attn_prefill(p, 1, 128, FAKE, FAKE, FAKE, NULL, FAKE, NULL, 0, NULL) == 3
+    assert lib.swa_attn_prefill(p, 1, 128, FAKE, FAKE, FAKE, NULL, FAKE, FAKE, 100, NULL) == 3
+    assert lib.swa_attn_prefill(p, 1, 128, FAKE, FAKE, FAKE, NULL, FAKE, FAKE + 16, 1 << 30, NULL) == 3
+    # empty inputs: nothing to do, nothing launched
+    assert lib.swa_attn_prefill(p, 0, 128, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0
+    assert lib.swa_attn_prefill(p, 2, 0, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0
+
+
+def test_decode_argument_errors(lib):
+    sl = _P(num_q_heads=96, num_kv_heads=8, window=512)
+    full = _P(num_q_heads=64, num_kv_heads=8, window=-1, rope_theta=5e6, rotary_dim=64)
+    args = lambda C, max_len: (FAKE, NULL, FAKE, FAKE, C, FAKE, max_len, FAKE, FAKE, 1 << 34, NULL)
+    assert lib.swa_attn_decode(sl, 4, *args(256, 100)) == 1             # ring capacity != W
+    assert lib.swa_attn_decode(full, 4, *args(1000, 2000)) == 1         # max_len > capacity
+    assert lib.swa_attn_decode(full, 4, *args(1000, 0)) == 1            # max_len < 1
+    assert lib.swa_attn_decode(_P(num_q_heads=34, num_kv_heads=2), 4, *args(64, 10)) == 2  # G > 16
+    a = list(args(4096, 4096))
+    a[0] = MIS
+    assert lib.swa_attn_decode(full, 4, *a) == 1
+    a = list(args(131072, 131072))
+    a[8] = NULL                                                         # workspace missing
+    assert lib.swa_attn_decode(full, 64, *a) == 3
+    assert lib.swa_attn_decode(sl, 0, *args(512, 512)) == 0              # empty batch
+
+
+def test_rope_argument_errors(lib):
+    p = _P(window=16)
+    assert lib.swa_rope_qk(p, 2, 4, FAKE, FAKE, NULL, 0, FAKE, FAKE, NULL, 16, NULL) == 1   # one cache only
+    assert lib.swa_rope_qk(p, 2, 4, FAKE, NULL, NULL, 0, FAKE, FAKE, FAKE, 16, NULL) == 1   # cache needs k
+    assert lib.swa_rope_qk(p, 2, 4, FAKE, FAKE, NULL, 0, FAKE, FAKE, FAKE, 8, NULL) == 1    # capacity != W
+    assert lib.swa_rope_qk(p, 2, 4, FAKE, FAKE, NULL, -1, NULL, NULL, NULL, 0, NULL) == 1   # negative pos0
+    assert lib.swa_rope_qk(p, 2, 4, MIS, FAKE, NULL, 0, NULL, NULL, NULL, 0, NULL) == 1
+    assert lib.swa_rope_qk(p, 0, 4, FAKE, FAKE, NULL, 0, NULL, NULL, NULL, 0, NULL) == 0
+    assert lib.swa_rope_qk(p, 2, 4, NULL, NULL, NULL, 0, NULL, NULL, NULL, 0, NULL) == 0

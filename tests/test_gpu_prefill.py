@@ -1,0 +1,122 @@
+"""swa_attn_prefill on the GPU against the oracle: the tiny case in full,
+window sweeps around tile edges, ragged lengths, partial / no RoPE, odd GQA
+groups, no gate, the uniform-score window-count probe at full size, and the
+full-size prefill workloads on seeded row samples."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from full_gqa_attention_swa_b200 import api, configs, inputs
+from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer, prefill_rows_sample
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(c):
+    return api.LayerParams(c.Hq, c.Hkv, 128, c.window, c.theta, c.rotary_dim)
+
+
+def _check_all_rows(cuda_device, p, B, S, seed, gate=True):
+    d = inputs.prefill_inputs(B, S, p.num_q_heads, p.num_kv_heads, 128, seed, with_gate=gate)
+    dev = {k: (None if t is None else t.to(cuda_device)) for k, t in d.items()}
+    out = api.attn_prefill(p, dev["q"], dev["k"], dev["v"], dev["gate"])
+    torch.cuda.synchronize()
+    ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]),
+                         None if d["gate"] is None else d["gate"].numpy())
+    return assert_close(out, ref, f"prefill B{B} S{S} W{p.window}")
+
+
+def test_tiny_config_all_rows(cuda_device):
+    c = configs.TINY
+    stats = _check_all_rows(cuda_device, _layer(c), c.B, c.S, c.seed)
+    assert stats["max_abs"] < 1e-2
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("W", [1, 2, 63, 64, 65, 127, 128, 129, 300, -1])
+def test_window_sweep(cuda_device, W):
+    p = api.LayerParams(4, 2, 128, W, 1e4, 128)
+    _check_all_rows(cuda_device, p, 1, 300, seed=100 + max(W, 0))
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("S", [1, 17, 128, 129, 255, 257, 640])
+@pytest.mark.parametrize("W", [64, -1])
+def test_ragged_lengths(cuda_device, S, W):
+    p = api.LayerParams(4, 1, 128, W, 1e4, 128)
+    _check_all_rows(cuda_device, p, 2, S, seed=200 + S)
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("theta,r", [(5e6, 64), (0.0, 128), (5e5, 32), (1e4, 6), (1e4, 0)])
+def test_rope_variants(cuda_device, theta, r):
+    p = api.LayerParams(8, 2, 128, 200, theta, r)
+    _check_all_rows(cuda_device, p, 1, 384, seed=300 + r)
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(6, 2), (2, 2), (3, 1), (16, 1)])
+def test_gqa_groups(cuda_device, Hq, Hkv):
+    p = api.LayerParams(Hq, Hkv, 128, 100, 1e4, 128)
+    _check_all_rows(cuda_device, p, 3, 200, seed=400 + Hq)
+    check_no_device_error()
+
+
+def test_no_gate_and_custom_scale(cuda_device):
+    _check_all_rows(cuda_device, api.LayerParams(4, 2, 128, 50, 1e4, 128), 2, 160, seed=501, gate=False)
+    _check_all_rows(cuda_device, api.LayerParams(4, 2, 128, -1, 1e4, 128, softmax_scale=0.05), 1, 200, seed=502)
+    check_no_device_error()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [configs.STEP_SLIDING, configs.MUSE_SLIDING], ids=lambda c: c.name)
+def test_uniform_score_probe_window_counts(cuda_device, cfg):
+    """Q = 0 makes every score 0: each output row is sigmoid(g) times the mean
+    of the visible values.  With one-hot values e_(j mod 128) every output dim
+    counts visible keys, so an off-by-one anywhere in the band shows, at the
+    full workload size."""
+    B, S = min(cfg.B, 2), cfg.S
+    p = _layer(cfg)
+    q = torch.zeros(B, S, cfg.Hq, 128, dtype=torch.bfloat16, device=cuda_device)
+    k = inputs.normal_bf16((B, S, cfg.Hkv, 128), cfg.seed, "k", cuda_device)
+    v = torch.zeros(B, S, cfg.Hkv, 128, dtype=torch.bfloat16, device=cuda_device)
+    j = torch.arange(S, device=cuda_device)
+    v[:, j, :, j % 128] = 1.0
+    gate = torch.zeros(B, S, cfg.Hq, device=cuda_device)
+    out = api.attn_prefill(p, q, k, v, gate)
+    torch.cuda.synchronize()
+    W = cfg.window
+    i = np.arange(S)
+    lo = np.maximum(0, i - W + 1)
+    n = i - lo + 1
+    # count of j in [lo, i] with j % 128 == d, for every d
+    d = np.arange(128)
+    def count_upto(x):  # number of j in [0, x) with j % 128 == d
+        return (x[:, None] // 128) + ((x[:, None] % 128) > d[None, :])
+    counts = count_upto(i + 1) - count_upto(lo)
+    expect = 0.5 * counts / n[:, None]                               # [S, 128]
+    got = out.float().cpu().numpy()                                  # [B,S,Hq,128]
+    # within one bf16 ulp: the kernel rounds 0.5/n and count*(0.5/n) in fp32
+    # before bf16; one key too many or too few moves the dim that gains or
+    # loses it by a whole count (>= 6% here)
+    e = np.broadcast_to(expect[None, :, None, :], got.shape)
+    bad = np.abs(got - e) > 2.0 ** -8 * np.abs(e)
+    assert not bad.any(), f"window count mismatch at {np.argwhere(bad)[:5].tolist()}"
+    check_no_device_error()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [configs.STEP_SLIDING, configs.STEP_FULL, configs.MUSE_SLIDING,
+                                 configs.MUSE_FULL], ids=lambda c: c.name)
+def test_full_size_sampled_rows(cuda_device, cfg):
+    p = _layer(cfg)
+    d = inputs.prefill_inputs(cfg.B, cfg.S, cfg.Hq, cfg.Hkv, 128, cfg.seed)
+    dev = {k: t.to(cuda_device) for k, t in d.items()}
+    out = api.attn_prefill(p, dev["q"], dev["k"], dev["v"], dev["gate"])
+    torch.cuda.synchronize()
+    rows = prefill_rows_sample(cfg.B, cfg.S, cfg.Hq, cfg.window, cfg.seed)
+    ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy(), rows=rows)
+    got = out.cpu()[torch.from_numpy(rows[:, 0]), torch.from_numpy(rows[:, 1]), torch.from_numpy(rows[:, 2])]
+    assert_close(got, ref, cfg.name)
+    check_no_device_error()
