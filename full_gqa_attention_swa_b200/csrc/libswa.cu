@@ -294,8 +294,9 @@ swa_status swa_attn_prefill(const swa_layer_params* p, int32_t B, int32_t S, con
     if (st != SWA_OK) return st;
     k_att = k_rot;
   }
-  CUtensorMap qm, km, vm;
+  CUtensorMap qm, km, vm, om;
   if ((st = encode_bshd(&qm, q, B, S, Hq, 128)) != SWA_OK) return st;
+  if ((st = encode_bshd(&om, out, B, S, Hq, 128)) != SWA_OK) return st;
   if ((st = encode_bshd(&km, k_att, B, S, Hkv, 128)) != SWA_OK) return st;
   if ((st = encode_bshd(&vm, v, B, S, Hkv, 128)) != SWA_OK) return st;
   swa::PrefillArgs a{};
@@ -304,10 +305,9 @@ swa_status swa_attn_prefill(const swa_layer_params* p, int32_t B, int32_t S, con
   a.scale_log2 = scale_log2(p);
   a.table = table;
   a.gate = gate;
-  a.out = out;
   a.n_q_tiles = (int)n_q_tiles;
   a.n_head_pairs = (G + 1) / 2;
-  st = cuda_status(swa::launch_prefill(a, qm, km, vm, s), "prefill launch");
+  st = cuda_status(swa::launch_prefill(a, qm, km, vm, om, s), "prefill launch");
   return st == SWA_OK ? ok() : st;
 }
 

@@ -12,9 +12,8 @@
 // dims per lane.  A lane reads its chunk and, for rotary dims, the partner
 // chunk rotary_dim/2 away, so both halves of a pair are read before any lane
 // of the row writes (a __syncwarp separates reads from writes when rotating in
-// place).  The angle is evaluated in fp64 (p up to 2^31, theta up to 5e6) and
-// its cos/sin rounded to fp32 once per (token, freq); each lane reuses them
-// across all heads it visits.
+// place).  Each lane forms cos/sin of its 8 frequencies once (see
+// rope_cos_sin) and reuses them across all heads it visits.
 #pragma once
 #include "swa_internal.cuh"
 
@@ -104,6 +103,20 @@ __device__ __forceinline__ void rotate_chunk(const uint16_t* row_src, uint16_t* 
   if (in_place) __syncwarp();
 }
 
+// cos and sin of a rotary angle.  The angle p * theta^(-2k/r) is formed in
+// fp64 and reduced to [-pi, pi] by subtracting the nearest multiple of 2*pi
+// (Cody-Waite reduction with 2*pi split into a double and its rounding
+// remainder), so its error stays near 1e-15 rad for any position below 2^31;
+// the reduced angle is then rounded to fp32 for sincosf.
+__device__ __forceinline__ void rope_cos_sin(double angle, float* c, float* s) {
+  const double kTwoPiHi = 6.283185307179586;       // 2*pi rounded to double
+  const double kTwoPiLo = 2.4492935982947064e-16;  // 2*pi - kTwoPiHi
+  const double n = rint(angle * (1.0 / kTwoPiHi));
+  double r = fma(-n, kTwoPiHi, angle);
+  r = fma(-n, kTwoPiLo, r);
+  sincosf((float)r, s, c);
+}
+
 // grid.x: ceil(B*S*16 / blockDim.x); grid.y: head split (heads h with
 // h % gridDim.y == blockIdx.y).
 __global__ void __launch_bounds__(256) rope_kernel(const RopeArgs a) {
@@ -122,10 +135,7 @@ __global__ void __launch_bounds__(256) rope_kernel(const RopeArgs a) {
   float c[8], s[8];
   for (int e = 0; e < 8; ++e) {
     if (L.role[e] != 0) {
-      double sd, cd;
-      sincos((double)p * a.inv_freq[L.freq[e]], &sd, &cd);
-      c[e] = (float)cd;
-      s[e] = (float)sd;
+      rope_cos_sin((double)p * a.inv_freq[L.freq[e]], &c[e], &s[e]);
     } else {
       c[e] = 1.f;
       s[e] = 0.f;

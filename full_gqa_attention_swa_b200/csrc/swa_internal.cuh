@@ -51,15 +51,14 @@ struct PrefillArgs {
   float scale_log2;          // softmax_scale * log2(e)
   const float2* table;       // [S][rotary_dim/2] cos/sin, when rotary_dim > 0
   const float* gate;         // [B,S,Hq] or nullptr
-  uint16_t* out;             // [B,S,Hq,D]
   int n_q_tiles;             // ceil(S / 128)
   int n_head_pairs;          // ceil(G / 2)
 };
 
-// q_map: 4-D {D, Hq, S, B}; k_map / v_map: 4-D {D, Hkv, S, B}; boxes
-// {64, 1, 128, 1}, 128-byte swizzle.
+// q_map / o_map: 4-D {D, Hq, S, B}; k_map / v_map: 4-D {D, Hkv, S, B};
+// boxes {64, 1, 128, 1}, 128-byte swizzle.
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                           const CUtensorMap& v_map, cudaStream_t stream);
+                           const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 
