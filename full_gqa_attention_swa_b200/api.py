@@ -25,7 +25,10 @@ STATUS_NAMES = {0: "SWA_OK", 1: "SWA_ERR_INVALID_ARG", 2: "SWA_ERR_UNSUPPORTED",
 # every function include/swa.h declares
 SYMBOLS = ("swa_rope_qk", "swa_prefill_workspace_size", "swa_attn_prefill", "swa_decode_workspace_size",
            "swa_attn_decode", "swa_kv_cache_bytes", "swa_status_string", "swa_last_error_detail",
-           "swa_device_error", "swa_version")
+           "swa_device_error", "swa_version", "swa_attn_decode_no_alloc")
+
+# bytes of the static device array behind swa_attn_decode_no_alloc
+NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class SwaError(RuntimeError):
@@ -98,6 +101,8 @@ def load(path: str = LIB_PATH):
     lib.swa_device_error.restype = ctypes.c_int
     lib.swa_version.argtypes = []
     lib.swa_version.restype = ctypes.c_char_p
+    lib.swa_attn_decode_no_alloc.argtypes = [P, i32, vp, vp, vp, vp, i32, vp, i32, vp, vp]
+    lib.swa_attn_decode_no_alloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -216,6 +221,28 @@ def attn_decode(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens, max_len
     _check(load().swa_attn_decode(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache), _ptr(v_cache), C,
                                   _ptr(seq_lens), int(max_len), _ptr(out), _ptr(workspace), nbytes,
                                   _stream(stream)))
+    return out
+
+
+def attn_decode_no_alloc(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens, max_len: int, out,
+                         stream=None):
+    """swa_attn_decode_no_alloc: attn_decode without a workspace, for callers
+    that cannot allocate device memory; the split-K partials live in a static
+    device array of NO_ALLOC_SCRATCH_BYTES inside libswa.so.  `out` must be
+    given (this call allocates nothing).  Calls that overlap on the GPU race
+    on the shared array."""
+    B = q.shape[0]
+    D = layer.head_dim
+    C = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (B, layer.num_q_heads, D))
+    _need(gate, "gate", torch.float32, (B, layer.num_q_heads))
+    _need(k_cache, "k_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(out, "out", torch.bfloat16, (B, layer.num_q_heads, D))
+    _check(load().swa_attn_decode_no_alloc(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache),
+                                           _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
+                                           _stream(stream)))
     return out
 
 

@@ -175,6 +175,67 @@ DecodePlan plan_decode(const swa_layer_params* p, int B, int max_len) {
   return pl;
 }
 
+// ------------------------------------------------ no-alloc decode scratch
+
+// Split-K partials of swa_attn_decode_no_alloc.  In host code this name is a
+// stand-in, not a device address: the kernels get the address that
+// cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) uint8_t g_decode_scratch[SWA_NO_ALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device, looked up once
+// per device (the first call on a device does this; it must not run under
+// stream capture).
+swa_status scratch_for_current_device(void** ptr) {
+  int dev = 0;
+  swa_status st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != SWA_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return fail(SWA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    st = cuda_status(cudaGetSymbolAddress(&p, g_decode_scratch), "cudaGetSymbolAddress(decode scratch)");
+    if (st != SWA_OK) return st;
+    g_scratch_ptr[dev] = p;
+  }
+  *ptr = g_scratch_ptr[dev];
+  return SWA_OK;
+}
+
+// The usual decode plan, or -- when its partials exceed the static array --
+// the same work in fewer, longer splits.
+swa_status plan_decode_no_alloc(const swa_layer_params* p, int B, int max_len, DecodePlan* out) {
+  DecodePlan pl = plan_decode(p, B, max_len);
+  if (pl.total <= SWA_NO_ALLOC_SCRATCH_BYTES) {
+    *out = pl;
+    return SWA_OK;
+  }
+  const long long kb = swa::kDecodeKeyBlock;
+  const long long n_vis = p->window > 0 ? (max_len < p->window ? max_len : p->window) : max_len;
+  const size_t rows = (size_t)B * p->num_q_heads;
+  const size_t per_split = rows * (kHeadDim * sizeof(float) + sizeof(float2));
+  // two 256-byte alignment pads between and after the two arrays
+  long long fit = (long long)((SWA_NO_ALLOC_SCRATCH_BYTES - 512) / per_split);
+  for (; fit >= 2; --fit) {
+    DecodePlan q{};
+    q.chunk = (int)(((n_vis + fit - 1) / fit + kb - 1) / kb * kb);
+    q.splits = (int)((n_vis + q.chunk - 1) / q.chunk);
+    q.o_bytes = round_up(rows * q.splits * kHeadDim * sizeof(float), 256);
+    q.ml_bytes = round_up(rows * q.splits * sizeof(float2), 256);
+    q.total = q.o_bytes + q.ml_bytes;
+    if (q.total <= SWA_NO_ALLOC_SCRATCH_BYTES) {
+      *out = q;
+      return SWA_OK;
+    }
+  }
+  return fail(SWA_ERR_UNSUPPORTED,
+              "no-alloc decode: %zu q-head rows need %zu bytes per split; the static scratch holds %u bytes",
+              rows, per_split, (unsigned)SWA_NO_ALLOC_SCRATCH_BYTES);
+}
+
 }  // namespace
 
 extern "C" {
@@ -357,6 +418,46 @@ swa_status swa_attn_decode(const swa_layer_params* p, int32_t B, const uint16_t*
   a.chunk = pl.chunk; a.max_splits = pl.splits;
   a.part_o = pl.splits > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
   a.part_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace) + pl.o_bytes) : nullptr;
+  st = cuda_status(swa::launch_decode(a, km, vm, (cudaStream_t)stream), "decode launch");
+  return st == SWA_OK ? ok() : st;
+}
+
+swa_status swa_attn_decode_no_alloc(const swa_layer_params* p, int32_t B, const uint16_t* q, const float* gate,
+                                    const uint16_t* k_cache, const uint16_t* v_cache, int32_t cache_capacity,
+                                    const int32_t* seq_lens, int32_t max_len, uint16_t* out, void* stream) {
+  swa_status st = check_layer(p);
+  if (st != SWA_OK) return st;
+  if (B < 0) return fail(SWA_ERR_INVALID_ARG, "B=%d must be >= 0", B);
+  if (B == 0) return ok();
+  const int Hq = p->num_q_heads, Hkv = p->num_kv_heads, G = Hq / Hkv;
+  if (G > 16) return fail(SWA_ERR_UNSUPPORTED, "decode supports up to 16 q-heads per kv-head (G=%d)", G);
+  if (!q || !k_cache || !v_cache || !seq_lens || !out)
+    return fail(SWA_ERR_INVALID_ARG, "q, k_cache, v_cache, seq_lens and out must be non-NULL");
+  const void* ptrs[] = {q, gate, k_cache, v_cache, seq_lens, out};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(SWA_ERR_INVALID_ARG, "tensor pointer %p is not 16-byte aligned", ptr);
+  if (cache_capacity < 1) return fail(SWA_ERR_INVALID_ARG, "cache_capacity=%d", cache_capacity);
+  if (p->window > 0 && cache_capacity != p->window)
+    return fail(SWA_ERR_INVALID_ARG, "sliding layer: cache_capacity=%d must equal window=%d", cache_capacity,
+                p->window);
+  if (max_len < 1) return fail(SWA_ERR_INVALID_ARG, "max_len=%d must be >= 1", max_len);
+  if (p->window < 0 && max_len > cache_capacity)
+    return fail(SWA_ERR_INVALID_ARG, "full layer: max_len=%d exceeds cache_capacity=%d", max_len, cache_capacity);
+  if ((long long)B * Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B*Hkv=%lld too large", (long long)B * Hkv);
+  DecodePlan pl;
+  if ((st = plan_decode_no_alloc(p, B, max_len, &pl)) != SWA_OK) return st;
+  void* scratch = nullptr;
+  if (pl.splits > 1 && (st = scratch_for_current_device(&scratch)) != SWA_OK) return st;
+  CUtensorMap km, vm;
+  if ((st = encode_cache(&km, k_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
+  if ((st = encode_cache(&vm, v_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
+  swa::DecodeArgs a{};
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.window = p->window; a.capacity = cache_capacity;
+  a.scale_log2 = scale_log2(p);
+  a.q = q; a.gate = gate; a.seq_lens = seq_lens; a.out = out;
+  a.chunk = pl.chunk; a.max_splits = pl.splits;
+  a.part_o = pl.splits > 1 ? reinterpret_cast<float*>(scratch) : nullptr;
+  a.part_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(scratch) + pl.o_bytes) : nullptr;
   st = cuda_status(swa::launch_decode(a, km, vm, (cudaStream_t)stream), "decode launch");
   return st == SWA_OK ? ok() : st;
 }

@@ -188,6 +188,47 @@ SWA_API swa_status swa_device_error(int32_t* code, int32_t reset);
 /* Library version string. */
 SWA_API const char* swa_version(void);
 
+/*
+ * swa_attn_decode_no_alloc -- swa_attn_decode for callers that cannot obtain
+ * device memory at call time.  The pages have no counterpart: this is an
+ * interface convenience of this library, not part of the method.
+ *
+ * Who needs it: code that runs where cudaMalloc is unavailable or unwanted,
+ * for example a plugin inside an engine that plans all device memory up
+ * front and hands its plugins no allocator, a host callback in which CUDA API
+ * calls are not permitted to allocate, or a latency-critical serving loop in
+ * which an allocation could stall on the device.  Such callers cannot supply
+ * the workspace that swa_attn_decode takes.
+ *
+ * Arguments and result are those of swa_attn_decode without the workspace:
+ * the split-K partial results live in one statically sized device array of
+ * SWA_NO_ALLOC_SCRATCH_BYTES bytes inside libswa.so, which every GPU that
+ * loads the library holds until the process exits.  Each split of a
+ * (sequence, q-head) row takes 520 bytes there.  When the usual split of the
+ * cache would not fit, fewer, longer splits are used; when even two splits
+ * per row do not fit (B * Hq * 2 * 520 bytes, plus 512 bytes of alignment,
+ * above SWA_NO_ALLOC_SCRATCH_BYTES) and the sequences need splitting, the call
+ * returns SWA_ERR_UNSUPPORTED and launches nothing.  Nothing in the array
+ * needs to start at zero: every partial a call reads was written earlier in
+ * the same call.
+ *
+ * All calls on a device share that array, and it keeps the contents of the
+ * last call: two calls whose kernels overlap on the GPU (different streams,
+ * or different host threads, without ordering between them) race on it and
+ * may return wrong results.  Order such calls on one stream or with events.
+ *
+ * The first call on each device does a one-time set-up (it looks up the
+ * device address of the array with cudaGetSymbolAddress while that device is
+ * current); make that first call before any stream capture.  The call itself
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define SWA_NO_ALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+SWA_API swa_status swa_attn_decode_no_alloc(const swa_layer_params* params, int32_t B, const uint16_t* q,
+                                            const float* gate, const uint16_t* k_cache, const uint16_t* v_cache,
+                                            int32_t cache_capacity, const int32_t* seq_lens, int32_t max_len,
+                                            uint16_t* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ def _P(**kw):
 
 def test_exports_every_declared_symbol(lib):
     declared = _declared()
-    assert len(declared) == len(api.SYMBOLS) == 10
+    assert len(declared) == len(api.SYMBOLS) == 11
     assert sorted(api.SYMBOLS) == declared
     for name in declared:
         assert hasattr(lib, name), name
