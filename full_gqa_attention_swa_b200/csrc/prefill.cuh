@@ -22,10 +22,12 @@
 //   warps 0-3   head slot 0: Q rotation, softmax (thread = query row)
 //   warps 4-7   head slot 1: same
 //   warps 8-11  O rescaling ("correction") and the epilogue (O/l * gate ->
-//               bf16 -> shared memory -> TMA store)
+//               bf16 -> shared memory, in the buffers the tile's last K and V
+//               tiles leave free)
 //   warp 12     tcgen05.mma issuer (one thread)
 //   warp 13     TMA producer (one thread)
-//   warps 14-15 idle
+//   warp 14     TMA store of the output tiles (one thread)
+//   warp 15     idle
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384)
 // O1 [384,512); P (bf16, two per column) overwrites the first 64 columns of
 // its S tile once the softmax has read S.
@@ -59,21 +61,20 @@ constexpr float kRescaleThreshold = 8.0f;       // log2 units
 // setmaxnreg split of the 128 x 512 registers the CTA is launched with
 constexpr uint32_t kRegsLaunch = 128;
 constexpr uint32_t kRegsSoftmax = 184;
-constexpr uint32_t kRegsCorrection = 96;
-constexpr uint32_t kRegsOther = 48;
+constexpr uint32_t kRegsCorrection = 88;
+constexpr uint32_t kRegsOther = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
 
 struct PrefillSmem {
   uint8_t q[2][kTileBytes];
   uint8_t kv[NKV][kTileBytes];
-  uint8_t ostage[kBoxBytes];  // one 64-dim half of an output tile
   float alpha[2][BM];
   float lsum[2][BM];
   uint64_t q_full[2], q_ready[2], q_empty[2];
   uint64_t kv_full[NKV], kv_empty[NKV];
   uint64_t s_full[2], p_full[2], alpha_full[2], o_ready[2], pv_done[2], l_full[2], l_empty[2];
-  uint64_t ost_full, ost_free;  // output staging buffer: written / free again
+  uint64_t ost_full[2], ost_empty[2];  // output tile staged / handed to the store warp
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -130,45 +131,45 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 }
 
 // Rotate one query row of a Q tile in shared memory (two 64-dim boxes with
-// 128-byte swizzle): pairs (k, k + r/2) for k < r/2, cos/sin from the table
-// row of this position.
-__device__ __forceinline__ void rotate_q_row(uint8_t* tile, int row, int r, const float2* __restrict__ cs) {
-  const int half = r / 2;
-  if ((half & 7) == 0) {
-    const float4* cs4 = reinterpret_cast<const float4*>(cs);
+// 128-byte swizzle): pairs (k, k + r/2) for k < r/2.  Vector form for
+// 16 | r: tb holds the (cos, sin) table row of this position as float4 =
+// two pairs, fetched before the tile arrives.
+__device__ __forceinline__ void rotate_q_row_vec(uint8_t* tile, int row, int half, const float4 (&tb)[32]) {
 #pragma unroll
-    for (int c0 = 0; c0 < 8; ++c0) {
-      if (c0 < half / 8) {
-        const int ea = c0 * 8, eb = ea + half;
-        uint4* pa = reinterpret_cast<uint4*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3));
-        uint4* pb = reinterpret_cast<uint4*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3));
-        uint4 A = *pa, Bv = *pb;
-        uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
-        uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
+  for (int c0 = 0; c0 < 8; ++c0) {
+    if (c0 * 8 < half) {
+      const int ea = c0 * 8, eb = ea + half;
+      uint4* pa = reinterpret_cast<uint4*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3));
+      uint4* pb = reinterpret_cast<uint4*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3));
+      uint4 A = *pa, Bv = *pb;
+      uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
+      uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float4 t = __ldg(cs4 + c0 * 4 + w);  // (cos, sin) of pairs ea+2w and ea+2w+1
-          const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
-          const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
-          a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
-          b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
-        }
-        *pa = A;
-        *pb = Bv;
+      for (int w = 0; w < 4; ++w) {
+        const float4 t = tb[c0 * 4 + w];  // (cos, sin) of pairs ea+2w and ea+2w+1
+        const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
+        const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
+        a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
+        b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
       }
+      *pa = A;
+      *pb = Bv;
     }
-  } else {
-    for (int k = 0; k < half; ++k) {
-      const int ea = k, eb = k + half;
-      uint16_t* pa = reinterpret_cast<uint16_t*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3)) +
-                     (ea & 7);
-      uint16_t* pb = reinterpret_cast<uint16_t*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3)) +
-                     (eb & 7);
-      const float x = __uint_as_float((uint32_t)*pa << 16), y = __uint_as_float((uint32_t)*pb << 16);
-      const float2 c = __ldg(cs + k);
-      *pa = __bfloat16_as_ushort(__float2bfloat16_rn(x * c.x - y * c.y));
-      *pb = __bfloat16_as_ushort(__float2bfloat16_rn(y * c.x + x * c.y));
-    }
+  }
+}
+
+// Element-wise form for any even r.
+__device__ __forceinline__ void rotate_q_row_scalar(uint8_t* tile, int row, int half, const float2* __restrict__ cs) {
+  for (int k = 0; k < half; ++k) {
+    const int ea = k, eb = k + half;
+    uint16_t* pa =
+        reinterpret_cast<uint16_t*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3)) + (ea & 7);
+    uint16_t* pb =
+        reinterpret_cast<uint16_t*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3)) + (eb & 7);
+    const float x = __uint_as_float((uint32_t)*pa << 16), y = __uint_as_float((uint32_t)*pb << 16);
+    const float2 c = __ldg(cs + k);
+    *pa = __bfloat16_as_ushort(__float2bfloat16_rn(x * c.x - y * c.y));
+    *pb = __bfloat16_as_ushort(__float2bfloat16_rn(y * c.x + x * c.y));
   }
 }
 
@@ -199,8 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kv_full[i], 1);
       mbar_init(&sm.kv_empty[i], 1);
     }
-    mbar_init(&sm.ost_full, BM);
-    mbar_init(&sm.ost_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.ost_full[i], BM);
+      mbar_init(&sm.ost_empty[i], 1);
+    }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -238,6 +241,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(sm.q[s], &q_map, &sm.q_full[s], 0, h, T.i0, T.b);
           tma_load_4d(sm.q[s] + kBoxBytes, &q_map, &sm.q_full[s], 64, h, T.i0, T.b);
           q_last[s] = it;
+        }
+        // warm L2 for the next tile of this CTA: its Q tiles (read once, from
+        // HBM, in 128-byte rows strided by Hq*256 bytes) and its cos/sin rows
+        if (t + (int)gridDim.x < n_tiles) {
+          const Tile N = decode_tile(a, t + gridDim.x);
+          for (int s = 0; s < 2; ++s) {
+            const int h = s ? N.h1 : N.h0;
+            tma_prefetch_4d(&q_map, 0, h, N.i0, N.b);
+            tma_prefetch_4d(&q_map, 64, h, N.i0, N.b);
+          }
+          if (a.rotary_dim > 0) {
+            const int rows = min(BM, a.S - N.i0);
+            const int half = a.rotary_dim / 2;
+            const uint32_t bytes = (uint32_t)(rows * half * sizeof(float2)) & ~15u;
+            if (bytes > 0) bulk_prefetch_l2(a.table + (size_t)N.i0 * half, bytes);
+          }
         }
         for (int u = 0; u < 2 * T.n_kv && ok; ++u) {
           const int g = kvt + u, buf = g % NKV, use = g / NKV;
@@ -332,7 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_ts(tmem + 384, tmem + 128 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                       (j > 0 || kk > 0));
             umma_commit(&sm.pv_done[1]);
-            umma_commit(&sm.kv_empty[gv % NKV]);
+            // the last K and V buffers of a tile stay with the epilogue, which
+            // stages the output there and hands them back after the store
+            if (more) umma_commit(&sm.kv_empty[gv % NKV]);
           }
           if (more) {
             const uint64_t kd = kvdesc0 + (uint64_t)(((gk % NKV) * kTileBytes) >> 4);
@@ -342,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_ss(tmem + 128, qdesc1 + off, kd + off, idesc_qk, kk > 0);
             }
             umma_commit(&sm.s_full[1]);
-            umma_commit(&sm.kv_empty[gk % NKV]);
+            if (j + 2 < n_kv) umma_commit(&sm.kv_empty[gk % NKV]);
             if (j + 2 == n_kv) umma_commit(&sm.q_empty[1]);
           }
         }
@@ -352,6 +373,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       // all MMAs issued by this thread complete before the CTA moves on
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, 200000000ull);
+    } else if (warp == 14 && lane == 0) {
+      // ========================================================== output store
+      // The epilogue stages head slot 0's output in the buffer of the tile's
+      // last K and slot 1's in that of its last V; this thread stores them
+      // with TMA and returns the buffers to the producer once read.
+      prefetch_tensormap(&o_map);
+      int it = 0, kvt = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+        const Tile T = decode_tile(a, t);
+        bool ok = true;
+        for (int s = 0; s < 2; ++s) {
+          if (!mbar_wait(&sm.ost_full[s], it & 1, abort_flag)) {
+            fail(abort_flag, kErrPrefill + 14);
+            ok = false;
+            break;
+          }
+          const int buf = (kvt + 2 * (T.n_kv - 1) + s) % NKV;
+          if (s == 0 || T.store1) {
+            const int h = s ? T.h1 : T.h0;
+            tma_store_4d(&o_map, sm.kv[buf], 0, h, T.i0, T.b);
+            tma_store_4d(&o_map, sm.kv[buf] + kBoxBytes, 64, h, T.i0, T.b);
+            bulk_commit_group();
+          }
+          mbar_arrive(&sm.ost_empty[s]);
+          bulk_wait_group_read0();
+          mbar_arrive(&sm.kv_empty[buf]);
+        }
+        if (!ok) break;
+        kvt += 2 * T.n_kv;
+      }
+      bulk_wait_group0();
     }
   } else if (warp < 8) {
     // ============================================================ softmax
@@ -365,13 +417,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile(a, t);
       const int i = T.i0 + row;
-      // ---- Q rotation of this slot's tile (rows beyond S stay zero)
+      // ---- Q rotation of this slot's tile (rows beyond S stay zero); the
+      // table row is fetched before the tile's arrival is awaited
+      const int half = a.rotary_dim / 2;
+      const bool rot = a.rotary_dim > 0 && i < a.S;
+      const bool vec = (half & 7) == 0;
+      float4 tb[32];
+      {
+        // rows without rotation read row 0; entries past half/2 repeat the last one
+        const float4* cs4 = reinterpret_cast<const float4*>(a.table + (size_t)(rot && vec ? i : 0) * half);
+        const int last = (rot && vec) ? half / 2 - 1 : 0;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) tb[k] = (rot && vec) ? __ldg(cs4 + min(k, last)) : make_float4(1.f, 0.f, 1.f, 0.f);
+      }
       if (!warp_wait(&sm.q_full[s], it & 1, abort_flag)) {
         fail(abort_flag, kErrPrefill + 6);
         break;
       }
-      if (a.rotary_dim > 0 && i < a.S)
-        rotate_q_row(sm.q[s], row, a.rotary_dim, a.table + (size_t)i * (a.rotary_dim / 2));
+      if (rot) {
+        if (vec)
+          rotate_q_row_vec(sm.q[s], row, half, tb);
+        else
+          rotate_q_row_scalar(sm.q[s], row, half, a.table + (size_t)i * half);
+      }
       fence_proxy_async_smem();
       mbar_arrive(&sm.q_ready[s]);
 
@@ -390,36 +458,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
         tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
         tmem_wait_ld();
-        const bool full_tile =
-            key0 + BN - 1 <= T.i0 && (a.window < 0 || key0 >= T.i0 + BM - 1 - a.window + 1);
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (full_tile) {
+        // which mask bounds cut this key tile (uniform over the tile):
+        // hi -- some key lies after some row (the diagonal tile);
+        // lo -- some key lies at or before row - W (the band's first tile)
+        const bool cut_hi = key0 + BN - 1 > T.i0;
+        const bool cut_lo = a.window > 0 && key0 < T.i0 + BM - a.window;
+        if (cut_hi || cut_lo) {
+          const int hi = cut_hi ? i - key0 : BN;                     // columns > hi are masked
+          const int lo = cut_lo ? i - a.window + 1 - key0 : -1;      // columns < lo are masked
 #pragma unroll
-          for (int e = 0; e < 128; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
-        } else {
-          // visible keys of this row inside the tile: columns [lo, hi]
-          const int hi = i - key0;
-          const int lo = a.window < 0 ? 0 : i - a.window + 1 - key0;
-#pragma unroll
-          for (int e = 0; e < 128; ++e) {
-            const float x = (e > hi || e < lo) ? -INFINITY : __uint_as_float(v[e]);
-            v[e] = __float_as_uint(x);
-            mx[e & 3] = fmaxf(mx[e & 3], x);
-          }
+          for (int e = 0; e < 128; ++e)
+            if (e > hi || e < lo) v[e] = __float_as_uint(-INFINITY);
         }
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int e = 0; e < 128; e += 2)
+          mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
         const float m_use = (mt - m > kRescaleThreshold) ? mt : m;  // m = -inf: always take mt
         const float m_safe = m_use == -INFINITY ? 0.f : m_use;
         const float alpha = fast_exp2(m - m_safe);
         sm.alpha[s][row] = alpha;
         mbar_arrive(&sm.alpha_full[s]);
-        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        // P = 2^(c S - m), two columns per packed FMA; masked columns give 0
+        const uint64_t cc = f2_pack(c, c), mm = f2_pack(-m_safe, -m_safe);
+        uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[64];
 #pragma unroll
         for (int e = 0; e < 128; e += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(v[e]), c, -m_safe));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), c, -m_safe));
-          sum[(e >> 1) & 3] += p0 + p1;
+          const uint64_t y = f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), cc, mm);
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+          sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(p0, p1));
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
@@ -427,7 +498,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[s]);
-        l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+        float s0, s1;
+        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
+        l = l * alpha + (s0 + s1);
         m = m_use;
       }
       if (!ok) break;
@@ -444,12 +517,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsCorrection>();
     const int row = threadIdx.x & (BM - 1);
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const bool leader = threadIdx.x == 256;
-    int it = 0, G = 0, su = 0;  // su: uses of the output staging buffer
+    int it = 0, G = 0, kvt = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile(a, t);
       const int i = T.i0 + row;
+      // gate logits of this row for both head slots, fetched early
+      float glog[2] = {0.f, 0.f};
+      if (a.gate && i < a.S) {
+        glog[0] = __ldg(a.gate + ((size_t)T.b * a.S + i) * a.Hq + T.h0);
+        glog[1] = __ldg(a.gate + ((size_t)T.b * a.S + i) * a.Hq + T.h1);
+      }
       for (int j = 0; j < T.n_kv && ok; ++j) {
         for (int s = 0; s < 2; ++s) {
           if (!warp_wait(&sm.alpha_full[s], (G + j) & 1, abort_flag)) {
@@ -484,10 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      // ---- epilogue: out = O / l * sigmoid(gate), staged for a TMA store
+      // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged for the store warp
       for (int s = 0; s < 2 && ok; ++s) {
         if (!warp_wait(&sm.pv_done[s], (G + T.n_kv - 1) & 1, abort_flag) ||
-            !warp_wait(&sm.l_full[s], it & 1, abort_flag)) {
+            !warp_wait(&sm.l_full[s], it & 1, abort_flag) ||
+            (it > 0 && !warp_wait(&sm.ost_empty[s], (it - 1) & 1, abort_flag))) {
           fail(abort_flag, kErrPrefill + 11);
           ok = false;
           break;
@@ -495,61 +574,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float l = sm.lsum[s][row];
         mbar_arrive(&sm.l_empty[s]);
-        const int h = s ? T.h1 : T.h0;
-        float g = 1.f;
-        if (a.gate && i < a.S) g = 1.f / (1.f + __expf(-__ldg(a.gate + ((size_t)T.b * a.S + i) * a.Hq + h)));
+        const float g = a.gate ? 1.f / (1.f + __expf(-glog[s])) : 1.f;
         const float f = g / l;
-        const bool store = s == 0 || T.store1;
+        // S_s(last) and P_s(last) are consumed, so this buffer is free: slot 0
+        // uses the last K tile's buffer, slot 1 the last V tile's
+        uint8_t* stage = sm.kv[(kvt + 2 * (T.n_kv - 1) + s) % NKV];
         const uint32_t oaddr = tmem + lane_off + 256 + s * 128;
-        for (int half = 0; half < 2; ++half) {
-          if (su > 0) {
-            // the previous store from the staging buffer has been read
-            if (leader) {
-              bulk_wait_group_read0();
-              mbar_arrive(&sm.ost_free);
-            }
-            if (!warp_wait(&sm.ost_free, (su - 1) & 1, abort_flag)) {
-              fail(abort_flag, kErrPrefill + 12);
-              ok = false;
-              break;
-            }
-          }
 #pragma unroll 1
-          for (int q2 = 0; q2 < 2; ++q2) {
-            uint32_t v[32];
-            tmem_ld32(oaddr + half * 64 + q2 * 32, v);
-            tmem_wait_ld();
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t v[32];
+          tmem_ld32(oaddr + q4 * 32, v);
+          tmem_wait_ld();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(v[8 * c4 + 0]) * f, __uint_as_float(v[8 * c4 + 1]) * f);
-              u.y = pack_bf16x2(__uint_as_float(v[8 * c4 + 2]) * f, __uint_as_float(v[8 * c4 + 3]) * f);
-              u.z = pack_bf16x2(__uint_as_float(v[8 * c4 + 4]) * f, __uint_as_float(v[8 * c4 + 5]) * f);
-              u.w = pack_bf16x2(__uint_as_float(v[8 * c4 + 6]) * f, __uint_as_float(v[8 * c4 + 7]) * f);
-              *reinterpret_cast<uint4*>(sm.ostage + sw128_off(row, q2 * 4 + c4)) = u;
-            }
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&sm.ost_full);
-          bool got = true;
-          if (leader) {
-            got = mbar_wait(&sm.ost_full, su & 1, abort_flag);
-            if (!got) fail(abort_flag, kErrPrefill + 13);
-            if (got && store) {
-              tma_store_4d(&o_map, sm.ostage, half * 64, h, T.i0, T.b);
-              bulk_commit_group();
-            }
-          }
-          ++su;
-          if (!__all_sync(0xffffffffu, got)) {
-            ok = false;
-            break;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int ch = q4 * 4 + c4;  // 16-byte chunk (8 dims) 0..15
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(v[8 * c4 + 0]) * f, __uint_as_float(v[8 * c4 + 1]) * f);
+            u.y = pack_bf16x2(__uint_as_float(v[8 * c4 + 2]) * f, __uint_as_float(v[8 * c4 + 3]) * f);
+            u.z = pack_bf16x2(__uint_as_float(v[8 * c4 + 4]) * f, __uint_as_float(v[8 * c4 + 5]) * f);
+            u.w = pack_bf16x2(__uint_as_float(v[8 * c4 + 6]) * f, __uint_as_float(v[8 * c4 + 7]) * f);
+            *reinterpret_cast<uint4*>(stage + (ch >> 3) * kBoxBytes + sw128_off(row, ch & 7)) = u;
           }
         }
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.ost_full[s]);
       }
       G += T.n_kv;
+      kvt += 2 * T.n_kv;
     }
-    if (leader) bulk_wait_group0();
   }
 
   tc_fence_before();
