@@ -300,6 +300,9 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--workload", default=configs.STEP_SLIDING.name, choices=sorted(configs.PREFILL))
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode_sliding", "decode_full"], default="all",
+                    help="run one leg only (profiling); prints that leg's own JSON line")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     c = configs.PREFILL[args.workload]
@@ -350,6 +353,19 @@ def main():
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
 
+    if args.only.startswith("decode"):
+        dc = configs.DECODE_SLIDING if args.only == "decode_sliding" else configs.DECODE_FULL
+        d_ms, nbytes = bench_decode(dc, max(args.steps, 1), max(args.warmup, 3), dev)
+        gbs = nbytes / (d_ms / 1e3) / 1e9
+        if rank == 0:
+            print(json.dumps({"metric": "decode HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": d_ms,
+                              "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                              "config": {"workload": dc.name},
+                              "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                           "frac": gbs / peaks["hbm_gbs"], "traffic": None}}), flush=True)
+        return
+
     ms, clocks, launches = bench_prefill(c, args.steps, max(args.warmup, 3), dev, dist)
     if dist is not None:
         t = torch.tensor([ms], device=dev)
@@ -369,12 +385,13 @@ def main():
                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
                         "peak_source": f"{peak_src} bf16 burst",
                         "kernel": "swa_attn_prefill (key-RoPE pre-pass + attention kernel), CUDA events"}
-    if rank == 0:
+    if rank == 0 and not args.no_e2e:
         e2e_steps = max(3, min(args.steps, 30))
         e_ms, h2d, d2h = bench_prefill_e2e(c, e2e_steps, dev)
         line["e2e"] = {"value": flops * e2e_steps / (e_ms / 1e3) / 1e12 * world, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-        if not args.no_decode:
+    if rank == 0:
+        if not args.no_decode and args.only == "all":
             extra = {}
             for dc in (configs.DECODE_SLIDING, configs.DECODE_FULL):
                 steps = 200 if dc.window > 0 else 10
@@ -383,9 +400,10 @@ def main():
                 extra[dc.name] = {"ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                                   "peak_source": f"{peak_src} hbm copy"}
             line["decode"] = extra
-        r, n, dt, thr = oracle_sample_rate(c, args.cpu_budget)
-        line["cpu_baseline"] = {"value": r, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-                                "sample": f"{n} seeded random (b, i, h) rows of {c.name}, {dt:.1f} s"}
+        if args.cpu_budget > 0:
+            r, n, dt, thr = oracle_sample_rate(c, args.cpu_budget)
+            line["cpu_baseline"] = {"value": r, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                    "sample": f"{n} seeded random (b, i, h) rows of {c.name}, {dt:.1f} s"}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
