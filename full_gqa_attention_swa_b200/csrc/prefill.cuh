@@ -22,22 +22,21 @@
 //   warps 0-3   head slot 0: Q rotation, softmax (thread = query row)
 //   warps 4-7   head slot 1: same
 //   warps 8-11  O rescaling ("correction") and the epilogue (O/l * gate ->
-//               bf16 -> shared memory, in the buffers the tile's last K and V
-//               tiles leave free)
+//               bf16 -> the slot's P buffer in shared memory)
 //   warp 12     tcgen05.mma issuer (one thread)
 //   warp 13     TMA producer (one thread)
 //   warp 14     TMA store of the output tiles (one thread)
 //   warp 15     idle
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384)
-// O1 [384,512); P (bf16, two per column) overwrites the first 64 columns of
-// its S tile once the softmax has read S.
+// O1 [384,512).  P (bf16) goes to a shared-memory buffer per head slot.
 //
 // Per key tile j and head slot s:
 //   MMA:     S_s = Q_s K_j^T            -> s_full[s]
-//   softmax: m, alpha, P_s -> TMEM      -> alpha_full[s], p_full[s]
+//   softmax: read S_s                   -> s_free[s] (S_s(j+1) may start)
+//            m, alpha, P_s -> smem      -> alpha_full[s], p_full[s]
 //   correct: wait PV_s(j-1), O_s *= alpha (skipped when alpha == 1 for the
 //            whole warp)                -> o_ready[s]
-//   MMA:     O_s += P_s V_j             -> pv_done[s]
+//   MMA:     O_s += P_s V_j             -> pv_done[s] (also frees p[s])
 // The max used for the exponentials only moves when the new row max exceeds
 // it by more than 8 (log2 units), so most tiles need no O rescale; exp2 of a
 // score then stays below 2^8, and the final normalisation by the row sum
@@ -51,7 +50,8 @@ namespace prefill_detail {
 
 constexpr int BM = 128;                         // query rows per tile
 constexpr int BN = 128;                         // keys per key tile
-constexpr int NKV = 4;                          // K/V ring buffers
+constexpr int NK = 2;                           // K tile ring
+constexpr int NV = 1;                           // V tile ring
 constexpr int kThreads = 512;
 constexpr uint32_t kBoxBytes = 128 * 128;       // 128 rows x 64 bf16
 constexpr uint32_t kTileBytes = 2 * kBoxBytes;  // 128 rows x 128 bf16
@@ -66,15 +66,21 @@ constexpr uint32_t kRegsOther = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
 
+// 231,712 bytes: within the 232,448-byte opt-in limit only because the
+// dynamic shared memory window starts 1024-byte aligned (checked at entry).
 struct PrefillSmem {
-  uint8_t q[2][kTileBytes];
-  uint8_t kv[NKV][kTileBytes];
+  uint8_t q[2][kTileBytes];    // Q of each head slot (rotated in place)
+  uint8_t p[2][kTileBytes];    // P (bf16) of each slot; also stages its output tile
+  uint8_t k[NK][kTileBytes];
+  uint8_t v[NV][kTileBytes];
   float alpha[2][BM];
   float lsum[2][BM];
   uint64_t q_full[2], q_ready[2], q_empty[2];
-  uint64_t kv_full[NKV], kv_empty[NKV];
-  uint64_t s_full[2], p_full[2], alpha_full[2], o_ready[2], pv_done[2], l_full[2], l_empty[2];
-  uint64_t ost_full[2], ost_empty[2];  // output tile staged / handed to the store warp
+  uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
+  uint64_t s_full[2], s_free[2], p_full[2], alpha_full[2], alpha_empty[2], o_ready[2], pv_done[2];
+  uint64_t l_full[2], l_empty[2];
+  uint64_t ost_full[2];  // output tile staged in p[s]
+  uint64_t pfree[2];     // the store of that tile has read p[s]
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -178,8 +184,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
                    const __grid_constant__ CUtensorMap o_map) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  PrefillSmem& sm =
-      *reinterpret_cast<PrefillSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // the 128-byte-swizzled tiles need 1024-byte alignment and the layout has
+  // no room to realign: leave (uniformly, before any barrier) if it is off
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) record_error(kErrPrefill + 15);
+    return;
+  }
+  PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = a.n_q_tiles * a.n_head_pairs * a.Hkv * a.B;
 
@@ -189,20 +200,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.q_ready[s], BM);
       mbar_init(&sm.q_empty[s], 1);
       mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_free[s], BM);
       mbar_init(&sm.p_full[s], BM);
       mbar_init(&sm.alpha_full[s], BM);
+      mbar_init(&sm.alpha_empty[s], BM);
       mbar_init(&sm.o_ready[s], BM);
       mbar_init(&sm.pv_done[s], 1);
       mbar_init(&sm.l_full[s], BM);
       mbar_init(&sm.l_empty[s], BM);
+      mbar_init(&sm.ost_full[s], BM);
+      mbar_init(&sm.pfree[s], 1);
     }
-    for (int i = 0; i < NKV; ++i) {
-      mbar_init(&sm.kv_full[i], 1);
-      mbar_init(&sm.kv_empty[i], 1);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.ost_full[i], BM);
-      mbar_init(&sm.ost_empty[i], 1);
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(&sm.v_full[i], 1);
+      mbar_init(&sm.v_empty[i], 1);
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -222,164 +237,182 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsOther>();
     if (warp == 13 && lane == 0) {
       // ========================================================== producer
+      // Per work tile: K(0), then [K(j+1), V(j)] per key tile (K runs one
+      // ahead, its 2-deep ring frees early; V's single buffer frees when both
+      // slots' P.V of the previous key tile complete).  The next tile's Q is
+      // loaded as soon as this tile's last QK^T has read Q.
       prefetch_tensormap(&q_map);
       prefetch_tensormap(&k_map);
       prefetch_tensormap(&v_map);
-      int it = 0, kvt = 0, issued_end = 0;
-      int q_last[2] = {-1, -1};  // tile index of the last Q load per slot
-      for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x, ++it) {
-        const Tile T = decode_tile(a, t);
-        bool ok = true;
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (it > 0 && !mbar_wait(&sm.q_empty[s], (it - 1) & 1, abort_flag)) {
-            fail(abort_flag, kErrPrefill + 1);
-            ok = false;
-            break;
-          }
+      int it = 0, kc = 0, vc = 0;           // tile counter, K / V loads issued
+      int k_end = 0, v_end = 0;             // loads issued (for the abort drain)
+      int q_last[2] = {-1, -1};
+      bool ok = true;
+      auto load_q = [&](int t_q, int it_q) -> bool {
+        const Tile N = decode_tile(a, t_q);
+        for (int s = 0; s < 2; ++s) {
+          if (it_q > 0 && !mbar_wait(&sm.q_empty[s], (it_q - 1) & 1, abort_flag)) return false;
           mbar_arrive_expect_tx(&sm.q_full[s], kTileBytes);
-          const int h = s ? T.h1 : T.h0;
-          tma_load_4d(sm.q[s], &q_map, &sm.q_full[s], 0, h, T.i0, T.b);
-          tma_load_4d(sm.q[s] + kBoxBytes, &q_map, &sm.q_full[s], 64, h, T.i0, T.b);
-          q_last[s] = it;
+          const int h = s ? N.h1 : N.h0;
+          tma_load_4d(sm.q[s], &q_map, &sm.q_full[s], 0, h, N.i0, N.b);
+          tma_load_4d(sm.q[s] + kBoxBytes, &q_map, &sm.q_full[s], 64, h, N.i0, N.b);
+          q_last[s] = it_q;
         }
-        // warm L2 for the next tile of this CTA: its Q tiles (read once, from
-        // HBM, in 128-byte rows strided by Hq*256 bytes) and its cos/sin rows
-        if (t + (int)gridDim.x < n_tiles) {
-          const Tile N = decode_tile(a, t + gridDim.x);
+        // warm L2 for the Q tiles and cos/sin rows of the tile after it
+        if (t_q + (int)gridDim.x < n_tiles) {
+          const Tile M = decode_tile(a, t_q + gridDim.x);
           for (int s = 0; s < 2; ++s) {
-            const int h = s ? N.h1 : N.h0;
-            tma_prefetch_4d(&q_map, 0, h, N.i0, N.b);
-            tma_prefetch_4d(&q_map, 64, h, N.i0, N.b);
+            const int h = s ? M.h1 : M.h0;
+            tma_prefetch_4d(&q_map, 0, h, M.i0, M.b);
+            tma_prefetch_4d(&q_map, 64, h, M.i0, M.b);
           }
           if (a.rotary_dim > 0) {
-            const int rows = min(BM, a.S - N.i0);
             const int half = a.rotary_dim / 2;
-            const uint32_t bytes = (uint32_t)(rows * half * sizeof(float2)) & ~15u;
-            if (bytes > 0) bulk_prefetch_l2(a.table + (size_t)N.i0 * half, bytes);
+            const uint32_t bytes = (uint32_t)(min(BM, a.S - M.i0) * half * sizeof(float2)) & ~15u;
+            if (bytes > 0) bulk_prefetch_l2(a.table + (size_t)M.i0 * half, bytes);
           }
         }
-        for (int u = 0; u < 2 * T.n_kv && ok; ++u) {
-          const int g = kvt + u, buf = g % NKV, use = g / NKV;
-          if (use > 0 && !mbar_wait(&sm.kv_empty[buf], (use - 1) & 1, abort_flag)) {
-            fail(abort_flag, kErrPrefill + 2);
-            ok = false;
-            break;
+        return true;
+      };
+      auto load_kv = [&](bool is_v, const Tile& T, int j) -> bool {
+        const int idx = is_v ? vc++ : kc++;
+        const int nb = is_v ? NV : NK;
+        const int buf = idx % nb, use = idx / nb;
+        uint64_t* full = is_v ? &sm.v_full[buf] : &sm.k_full[buf];
+        uint64_t* empty = is_v ? &sm.v_empty[buf] : &sm.k_empty[buf];
+        if (use > 0 && !mbar_wait(empty, (use - 1) & 1, abort_flag)) return false;
+        uint8_t* dst = is_v ? sm.v[buf] : sm.k[buf];
+        const CUtensorMap* map = is_v ? &v_map : &k_map;
+        const int key0 = (T.kt_lo + j) * BN;
+        mbar_arrive_expect_tx(full, kTileBytes);
+        tma_load_4d(dst, map, full, 0, T.kvh, key0, T.b);
+        tma_load_4d(dst + kBoxBytes, map, full, 64, T.kvh, key0, T.b);
+        if (is_v) {
+          v_end = idx + 1;
+          if (j + 1 < T.n_kv) {  // the next V comes through L2
+            tma_prefetch_4d(&v_map, 0, T.kvh, key0 + BN, T.b);
+            tma_prefetch_4d(&v_map, 64, T.kvh, key0 + BN, T.b);
           }
-          mbar_arrive_expect_tx(&sm.kv_full[buf], kTileBytes);
-          const int key0 = (T.kt_lo + (u >> 1)) * BN;
-          const CUtensorMap* map = (u & 1) ? &v_map : &k_map;
-          tma_load_4d(sm.kv[buf], map, &sm.kv_full[buf], 0, T.kvh, key0, T.b);
-          tma_load_4d(sm.kv[buf] + kBoxBytes, map, &sm.kv_full[buf], 64, T.kvh, key0, T.b);
-          issued_end = g + 1;
+        } else {
+          k_end = idx + 1;
         }
-        kvt += 2 * T.n_kv;
+        return true;
+      };
+      if (blockIdx.x < (unsigned)n_tiles && !load_q(blockIdx.x, 0)) ok = false;
+      for (int t = blockIdx.x; t < n_tiles && ok && !*abort_flag; t += gridDim.x, ++it) {
+        const Tile T = decode_tile(a, t);
+        const bool has_next = t + (int)gridDim.x < n_tiles;
+        for (int j = -1; j < T.n_kv && ok; ++j) {
+          if (j + 1 < T.n_kv) ok = load_kv(false, T, j + 1);
+          if (ok && j >= 0) {
+            // the next tile's Q waits for this tile's last QK^T: issue it
+            // before the last V (which waits for the previous P.V), or after
+            // the only V of a one-key-tile tile
+            const bool last = j == T.n_kv - 1;
+            if (last && has_next && T.n_kv >= 2) ok = load_q(t + gridDim.x, it + 1);
+            if (ok) ok = load_kv(true, T, j);
+            if (ok && last && has_next && T.n_kv == 1) ok = load_q(t + gridDim.x, it + 1);
+          }
+        }
+        if (!ok) fail(abort_flag, kErrPrefill + 1);
       }
       if (*abort_flag) {
         // let every copy this thread started land before the CTA exits
         for (int s = 0; s < 2; ++s)
           if (q_last[s] >= 0) mbar_wait(&sm.q_full[s], q_last[s] & 1, nullptr, 200000000ull);
-        for (int g = issued_end > NKV ? issued_end - NKV : 0; g < issued_end; ++g)
-          mbar_wait(&sm.kv_full[g % NKV], (g / NKV) & 1, nullptr, 200000000ull);
+        for (int g = k_end > NK ? k_end - NK : 0; g < k_end; ++g)
+          mbar_wait(&sm.k_full[g % NK], (g / NK) & 1, nullptr, 200000000ull);
+        for (int g = v_end > NV ? v_end - NV : 0; g < v_end; ++g)
+          mbar_wait(&sm.v_full[g % NV], (g / NV) & 1, nullptr, 200000000ull);
       }
     } else if (warp == 12 && lane == 0) {
       // ========================================================== MMA issuer
-      // Descriptors advance by adding (byte offset >> 4) to the start-address
-      // field; every tile here sits below 256 KB of shared memory, so the
-      // 14-bit field never carries.
+      // In-phase order per key tile: [S_0(j+1), S_1(j+1)] then [O_0 += P_0 V_j,
+      // O_1 += P_1 V_j], each pair issued one MMA of each GEMM in turn.  S(j+1)
+      // needs only that the softmax has read S(j) (P is in shared memory), so
+      // both QK^T of the next key tile overlap the softmax and the P.V of the
+      // current one: up to four independent accumulation chains in the pipe,
+      // where a lone chain of dependent tcgen05.mma runs at a fraction of its
+      // rate.  Descriptors advance by adding (byte offset >> 4) to the
+      // start-address field (no carry below 256 KB).
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, 128, false, true);
-      const uint64_t qdesc0 = sw128_desc(smem_u32(sm.q[0]), 16, 1024);
-      const uint64_t qdesc1 = sw128_desc(smem_u32(sm.q[1]), 16, 1024);
-      const uint64_t kvdesc0 = sw128_desc(smem_u32(sm.kv[0]), 16, 1024);
-      const uint64_t vdesc0 = sw128_desc(smem_u32(sm.kv[0]), kBoxBytes, 1024);
-      int it = 0, G = 0, kvt = 0;
+      const uint64_t qd0 = sw128_desc(smem_u32(sm.q[0]), 16, 1024), qd1 = sw128_desc(smem_u32(sm.q[1]), 16, 1024);
+      const uint64_t pd0 = sw128_desc(smem_u32(sm.p[0]), 16, 1024), pd1 = sw128_desc(smem_u32(sm.p[1]), 16, 1024);
+      const uint64_t kdesc0 = sw128_desc(smem_u32(sm.k[0]), 16, 1024);
+      const uint64_t vdesc0 = sw128_desc(smem_u32(sm.v[0]), kBoxBytes, 1024);
+      int it = 0, G = 0, kc = 0, vc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
         const int n_kv = decode_tile(a, t).n_kv;
-        ok = mbar_wait(&sm.q_ready[0], it & 1, abort_flag) && mbar_wait(&sm.q_ready[1], it & 1, abort_flag) &&
-             mbar_wait(&sm.kv_full[kvt % NKV], (kvt / NKV) & 1, abort_flag);
-        if (!ok) {
+        if (!mbar_wait(&sm.q_ready[0], it & 1, abort_flag) || !mbar_wait(&sm.q_ready[1], it & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 3);
+          ok = false;
           break;
         }
-        tc_fence_after();
-        for (int j = -1; j < n_kv; ++j) {
-          // j == -1: the first S tiles of this work tile; then PV(j) and S(j+1)
-          const int gv = kvt + 2 * j + 1, gk = kvt + 2 * j + 2;
-          const bool more = j + 1 < n_kv;
-          const uint32_t ph = (G + j) & 1;
-          if (j >= 0) {
-            ok = mbar_wait(&sm.kv_full[gv % NKV], (gv / NKV) & 1, abort_flag) &&
-                 mbar_wait(&sm.p_full[0], ph, abort_flag) && mbar_wait(&sm.o_ready[0], ph, abort_flag);
+        for (int j = -1; j < n_kv && ok; ++j) {
+          if (j + 1 < n_kv) {
+            const int g1 = G + j + 1, ki = kc + j + 1;
+            ok = (g1 == 0 || (mbar_wait(&sm.s_free[0], (g1 - 1) & 1, abort_flag) &&
+                              mbar_wait(&sm.s_free[1], (g1 - 1) & 1, abort_flag))) &&
+                 mbar_wait(&sm.k_full[ki % NK], (ki / NK) & 1, abort_flag);
             if (!ok) {
               fail(abort_flag, kErrPrefill + 4);
               break;
             }
             tc_fence_after();
-            const uint64_t vd = vdesc0 + (uint64_t)(((gv % NKV) * kTileBytes) >> 4);
-#pragma unroll 1
-            for (int kk = 0; kk < 8; ++kk)
-              umma_ts(tmem + 256, tmem + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv, (j > 0 || kk > 0));
-            umma_commit(&sm.pv_done[0]);
-          }
-          if (more) {
-            if (j >= 0 && !mbar_wait(&sm.kv_full[gk % NKV], (gk / NKV) & 1, abort_flag)) {
-              fail(abort_flag, kErrPrefill + 4);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t kd = kvdesc0 + (uint64_t)(((gk % NKV) * kTileBytes) >> 4);
+            const uint64_t kd = kdesc0 + (uint64_t)(((ki % NK) * kTileBytes) >> 4);
 #pragma unroll 1
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t off = (uint64_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
-              umma_ss(tmem, qdesc0 + off, kd + off, idesc_qk, kk > 0);
+              umma_ss(tmem, qd0 + off, kd + off, idesc_qk, kk > 0);
+              umma_ss(tmem + 128, qd1 + off, kd + off, idesc_qk, kk > 0);
             }
             umma_commit(&sm.s_full[0]);
-            if (j + 2 == n_kv) umma_commit(&sm.q_empty[0]);
+            umma_commit(&sm.s_full[1]);
+            umma_commit(&sm.k_empty[ki % NK]);
+            if (j + 2 == n_kv) {
+              umma_commit(&sm.q_empty[0]);
+              umma_commit(&sm.q_empty[1]);
+            }
           }
           if (j >= 0) {
-            if (!mbar_wait(&sm.p_full[1], ph, abort_flag) || !mbar_wait(&sm.o_ready[1], ph, abort_flag)) {
+            const int g = G + j, vi = vc + j;
+            ok = mbar_wait(&sm.p_full[0], g & 1, abort_flag) && mbar_wait(&sm.o_ready[0], g & 1, abort_flag) &&
+                 mbar_wait(&sm.p_full[1], g & 1, abort_flag) && mbar_wait(&sm.o_ready[1], g & 1, abort_flag) &&
+                 mbar_wait(&sm.v_full[vi % NV], (vi / NV) & 1, abort_flag);
+            if (!ok) {
               fail(abort_flag, kErrPrefill + 5);
-              ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t vd = vdesc0 + (uint64_t)(((gv % NKV) * kTileBytes) >> 4);
-#pragma unroll 1
-            for (int kk = 0; kk < 8; ++kk)
-              umma_ts(tmem + 384, tmem + 128 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
-                      (j > 0 || kk > 0));
-            umma_commit(&sm.pv_done[1]);
-            // the last K and V buffers of a tile stay with the epilogue, which
-            // stages the output there and hands them back after the store
-            if (more) umma_commit(&sm.kv_empty[gv % NKV]);
-          }
-          if (more) {
-            const uint64_t kd = kvdesc0 + (uint64_t)(((gk % NKV) * kTileBytes) >> 4);
+            const uint64_t vd = vdesc0 + (uint64_t)(((vi % NV) * kTileBytes) >> 4);
 #pragma unroll 1
             for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t off = (uint64_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
-              umma_ss(tmem + 128, qdesc1 + off, kd + off, idesc_qk, kk > 0);
+              const uint64_t aoff = (uint64_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
+              const uint64_t boff = (uint64_t)((kk * 2048) >> 4);
+              const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+              umma_ss(tmem + 256, pd0 + aoff, vd + boff, idesc_pv, acc);
+              umma_ss(tmem + 384, pd1 + aoff, vd + boff, idesc_pv, acc);
             }
-            umma_commit(&sm.s_full[1]);
-            if (j + 2 < n_kv) umma_commit(&sm.kv_empty[gk % NKV]);
-            if (j + 2 == n_kv) umma_commit(&sm.q_empty[1]);
+            umma_commit(&sm.pv_done[0]);
+            umma_commit(&sm.pv_done[1]);
+            umma_commit(&sm.v_empty[vi % NV]);
           }
         }
         G += n_kv;
-        kvt += 2 * n_kv;
+        kc += n_kv;
+        vc += n_kv;
       }
       // all MMAs issued by this thread complete before the CTA moves on
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, 200000000ull);
     } else if (warp == 14 && lane == 0) {
       // ========================================================== output store
-      // The epilogue stages head slot 0's output in the buffer of the tile's
-      // last K and slot 1's in that of its last V; this thread stores them
-      // with TMA and returns the buffers to the producer once read.
+      // The epilogue stages each slot's output tile in that slot's P buffer;
+      // this thread stores it with TMA and frees the buffer once it is read.
       prefetch_tensormap(&o_map);
-      int it = 0, kvt = 0;
+      int it = 0;
       for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
         const Tile T = decode_tile(a, t);
         bool ok = true;
@@ -389,19 +422,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const int buf = (kvt + 2 * (T.n_kv - 1) + s) % NKV;
           if (s == 0 || T.store1) {
             const int h = s ? T.h1 : T.h0;
-            tma_store_4d(&o_map, sm.kv[buf], 0, h, T.i0, T.b);
-            tma_store_4d(&o_map, sm.kv[buf] + kBoxBytes, 64, h, T.i0, T.b);
+            tma_store_4d(&o_map, sm.p[s], 0, h, T.i0, T.b);
+            tma_store_4d(&o_map, sm.p[s] + kBoxBytes, 64, h, T.i0, T.b);
             bulk_commit_group();
           }
-          mbar_arrive(&sm.ost_empty[s]);
           bulk_wait_group_read0();
-          mbar_arrive(&sm.kv_empty[buf]);
+          mbar_arrive(&sm.pfree[s]);
         }
         if (!ok) break;
-        kvt += 2 * T.n_kv;
       }
       bulk_wait_group0();
     }
@@ -458,6 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
         tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&sm.s_free[s]);  // S_s may be overwritten by the next QK^T
         // which mask bounds cut this key tile (uniform over the tile):
         // hi -- some key lies after some row (the diagonal tile);
         // lo -- some key lies at or before row - W (the band's first tile)
@@ -478,6 +510,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_use = (mt - m > kRescaleThreshold) ? mt : m;  // m = -inf: always take mt
         const float m_safe = m_use == -INFINITY ? 0.f : m_use;
         const float alpha = fast_exp2(m - m_safe);
+        // the correction has read the previous alpha (the softmax can run a
+        // key tile ahead of it now that S(j+1) no longer waits for P(j).V)
+        if (G + j > 0 && !warp_wait(&sm.alpha_empty[s], (G + j - 1) & 1, abort_flag)) {
+          fail(abort_flag, kErrPrefill + 17);
+          ok = false;
+          break;
+        }
         sm.alpha[s][row] = alpha;
         mbar_arrive(&sm.alpha_full[s]);
         // P = 2^(c S - m), two columns per packed FMA; masked columns give 0
@@ -493,10 +532,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(p0, p1));
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
-        tmem_st32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
-        tmem_wait_st();
-        tc_fence_before();
+        // p[s] is free once P_s(j-1).V has completed; at a tile's first key
+        // tile it holds the previous tile's output until the store has read
+        // it.  (S(j) completing implies P(j-2).V completed, since its commit
+        // covers every earlier MMA, so these waits are never two phases ahead.)
+        if (j > 0 ? !warp_wait(&sm.pv_done[s], (G + j - 1) & 1, abort_flag)
+                  : (it > 0 && !warp_wait(&sm.pfree[s], (it - 1) & 1, abort_flag))) {
+          fail(abort_flag, kErrPrefill + 16);
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch)
+          *reinterpret_cast<uint4*>(sm.p[s] + (ch >> 3) * kBoxBytes + sw128_off(row, ch & 7)) =
+              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        fence_proxy_async_smem();
         mbar_arrive(&sm.p_full[s]);
         float s0, s1;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
@@ -517,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsCorrection>();
     const int row = threadIdx.x & (BM - 1);
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    int it = 0, G = 0, kvt = 0;
+    int it = 0, G = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile(a, t);
@@ -536,6 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const float alpha = sm.alpha[s][row];
+          mbar_arrive(&sm.alpha_empty[s]);
           if (j > 0) {
             if (!warp_wait(&sm.pv_done[s], (G + j - 1) & 1, abort_flag)) {
               fail(abort_flag, kErrPrefill + 10);
@@ -562,11 +613,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged for the store warp
+      // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged in p[s] for
+      // the store warp (P_s(last) is consumed once that slot's P.V is done)
       for (int s = 0; s < 2 && ok; ++s) {
         if (!warp_wait(&sm.pv_done[s], (G + T.n_kv - 1) & 1, abort_flag) ||
-            !warp_wait(&sm.l_full[s], it & 1, abort_flag) ||
-            (it > 0 && !warp_wait(&sm.ost_empty[s], (it - 1) & 1, abort_flag))) {
+            !warp_wait(&sm.l_full[s], it & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 11);
           ok = false;
           break;
@@ -576,9 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.l_empty[s]);
         const float g = a.gate ? 1.f / (1.f + __expf(-glog[s])) : 1.f;
         const float f = g / l;
-        // S_s(last) and P_s(last) are consumed, so this buffer is free: slot 0
-        // uses the last K tile's buffer, slot 1 the last V tile's
-        uint8_t* stage = sm.kv[(kvt + 2 * (T.n_kv - 1) + s) % NKV];
+        uint8_t* stage = sm.p[s];
         const uint32_t oaddr = tmem + lane_off + 256 + s * 128;
 #pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -600,7 +649,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.ost_full[s]);
       }
       G += T.n_kv;
-      kvt += 2 * T.n_kv;
     }
   }
 
@@ -620,7 +668,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const
   const long long n_tiles = (long long)a.n_q_tiles * a.n_head_pairs * a.Hkv * a.B;
   if (n_tiles == 0) return cudaSuccess;
   if (n_tiles > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  const size_t smem = sizeof(PrefillSmem) + 1024;
+  const size_t smem = sizeof(PrefillSmem);
   static int n_sm = 0;
   static bool checked = false;
   if (!checked) {
