@@ -139,7 +139,7 @@ PrefillPlan plan_prefill(const swa_layer_params* p, int B, int S) {
   pl.rotate = rotates(p);
   if (pl.rotate) {
     pl.k_bytes = round_up((size_t)B * S * p->num_kv_heads * kHeadDim * 2, 256);
-    pl.table_bytes = round_up((size_t)S * (p->rotary_dim / 2) * sizeof(float2), 256);
+    pl.table_bytes = round_up((size_t)swa::rope_table_bytes(S, p->rotary_dim / 2), 256);
   }
   pl.total = pl.k_bytes + pl.table_bytes;
   return pl;

@@ -19,10 +19,11 @@
 // output store of neighbouring tiles overlap with the tensor-core work.
 //
 // Warp roles (16 warps, registers rebalanced with setmaxnreg):
-//   warps 0-3   head slot 0: Q rotation, softmax (thread = query row)
+//   warps 0-3   head slot 0: softmax (thread = query row)
 //   warps 4-7   head slot 1: same
-//   warps 8-11  O rescaling ("correction") and the epilogue (O/l * gate ->
-//               bf16 -> the slot's P buffer in shared memory)
+//   warps 8-11  O rescaling ("correction"), the RoPE of the next tile's Q
+//               (both slots) and the epilogue (O/l * gate -> bf16 -> the
+//               slot's P buffer in shared memory)
 //   warp 12     tcgen05.mma issuer (one thread)
 //   warp 13     TMA producer (one thread)
 //   warp 14     TMA store of the output tiles (one thread)
@@ -32,11 +33,17 @@
 //
 // Per key tile j and head slot s:
 //   MMA:     S_s = Q_s K_j^T            -> s_full[s]
-//   softmax: read S_s                   -> s_free[s] (S_s(j+1) may start)
-//            m, alpha, P_s -> smem      -> alpha_full[s], p_full[s]
+//   softmax: read S_s                   -> s_free (both slots: S(j+1) may start)
+//            m, alpha                   -> alpha_full[s]
+//            P_s = 2^(S_s - m) -> smem  -> pv_ready
 //   correct: wait PV_s(j-1), O_s *= alpha (skipped when alpha == 1 for the
-//            whole warp)                -> o_ready[s]
+//            whole warp)                -> pv_ready
 //   MMA:     O_s += P_s V_j             -> pv_done[s] (also frees p[s])
+// The MMA thread waits on one barrier per hand-off (s_free, pv_ready) rather
+// than one per slot and producer: each wait is a shared-memory round trip that
+// queues behind the softmax warps' SFU traffic on the same sub-partition.
+// The exponentials run on the SFU (a polynomial path on the FMA pipe exists,
+// see poly_column_pair).
 // The max used for the exponentials only moves when the new row max exceeds
 // it by more than 8 (log2 units), so most tiles need no O rescale; exp2 of a
 // score then stays below 2^8, and the final normalisation by the row sum
@@ -75,9 +82,12 @@ struct PrefillSmem {
   uint8_t v[NV][kTileBytes];
   float alpha[2][BM];
   float lsum[2][BM];
-  uint64_t q_full[2], q_ready[2], q_empty[2];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t q_ready;  // both slots' Q rotated (128 arrivals)
   uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
-  uint64_t s_full[2], s_free[2], p_full[2], alpha_full[2], alpha_empty[2], o_ready[2], pv_done[2];
+  uint64_t s_full[2], alpha_full[2], alpha_empty[2], pv_done[2];
+  uint64_t s_free;    // both slots have read S (256 arrivals)
+  uint64_t pv_ready;  // both slots' P written and O rescaled (512 arrivals)
   uint64_t l_full[2], l_empty[2];
   uint64_t ost_full[2];  // output tile staged in p[s]
   uint64_t pfree[2];     // the store of that tile has read p[s]
@@ -111,6 +121,14 @@ __device__ __forceinline__ Tile decode_tile(const PrefillArgs& a, int t) {
   return T;
 }
 
+// Column pairs (of every 8) whose exponentials run on the FMA pipe
+// (exp2_poly2) instead of the SFU.  Zero: the step is bound by the tensor
+// pipe and the MMA thread's hand-offs, not by the SFU, and the polynomial's
+// extra issue slots on the MMA thread's sub-partition slow it (by 5-8% at 3 of
+// 8 pairs).
+constexpr int kPolyPairsPer8 = 0;
+__host__ __device__ constexpr bool poly_column_pair(int pair) { return (pair & 7) < kPolyPairsPer8; }
+
 __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
@@ -136,46 +154,56 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// Rotate one query row of a Q tile in shared memory (two 64-dim boxes with
-// 128-byte swizzle): pairs (k, k + r/2) for k < r/2.  Vector form for
-// 16 | r: tb holds the (cos, sin) table row of this position as float4 =
-// two pairs, fetched before the tile arrives.
-__device__ __forceinline__ void rotate_q_row_vec(uint8_t* tile, int row, int half, const float4 (&tb)[32]) {
+// Rotate query row `row` (position i) of both head slots' Q tiles in shared
+// memory (two 64-dim boxes each, 128-byte swizzle): pairs (k, k + r/2) for
+// k < r/2.  Vector form for 16 | r: per 8-dim chunk, four 16-byte table
+// slices (two pairs each) that the warp's 32 rows load from 512 contiguous
+// bytes apiece.
+__device__ __forceinline__ void rotate_q_rows_vec(uint8_t* q0, uint8_t* q1, int row, int half,
+                                                  const float4* __restrict__ tgroup) {
+#pragma unroll 1
+  for (int c0 = 0; c0 < half / 8; ++c0) {
+    const int ea = c0 * 8, eb = ea + half;
+    float4 t[4];
 #pragma unroll
-  for (int c0 = 0; c0 < 8; ++c0) {
-    if (c0 * 8 < half) {
-      const int ea = c0 * 8, eb = ea + half;
-      uint4* pa = reinterpret_cast<uint4*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3));
-      uint4* pb = reinterpret_cast<uint4*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3));
-      uint4 A = *pa, Bv = *pb;
+    for (int w = 0; w < 4; ++w) t[w] = __ldg(tgroup + (size_t)(c0 * 4 + w) * 32);  // pairs ea+2w, ea+2w+1
+    const uint32_t oa = (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3);
+    const uint32_t ob = (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3);
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      uint8_t* tile = s ? q1 : q0;
+      uint4 A = *reinterpret_cast<uint4*>(tile + oa), Bv = *reinterpret_cast<uint4*>(tile + ob);
       uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
       uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const float4 t = tb[c0 * 4 + w];  // (cos, sin) of pairs ea+2w and ea+2w+1
         const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
         const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
-        a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
-        b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
+        a32[w] = pack_bf16x2(x0 * t[w].x - y0 * t[w].y, x1 * t[w].z - y1 * t[w].w);
+        b32[w] = pack_bf16x2(y0 * t[w].x + x0 * t[w].y, y1 * t[w].z + x1 * t[w].w);
       }
-      *pa = A;
-      *pb = Bv;
+      *reinterpret_cast<uint4*>(tile + oa) = A;
+      *reinterpret_cast<uint4*>(tile + ob) = Bv;
     }
   }
 }
 
 // Element-wise form for any even r.
-__device__ __forceinline__ void rotate_q_row_scalar(uint8_t* tile, int row, int half, const float2* __restrict__ cs) {
+__device__ __forceinline__ void rotate_q_rows_scalar(uint8_t* q0, uint8_t* q1, int row, int i, int half,
+                                                     const float2* __restrict__ table) {
   for (int k = 0; k < half; ++k) {
     const int ea = k, eb = k + half;
-    uint16_t* pa =
-        reinterpret_cast<uint16_t*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3)) + (ea & 7);
-    uint16_t* pb =
-        reinterpret_cast<uint16_t*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3)) + (eb & 7);
-    const float x = __uint_as_float((uint32_t)*pa << 16), y = __uint_as_float((uint32_t)*pb << 16);
-    const float2 c = __ldg(cs + k);
-    *pa = __bfloat16_as_ushort(__float2bfloat16_rn(x * c.x - y * c.y));
-    *pb = __bfloat16_as_ushort(__float2bfloat16_rn(y * c.x + x * c.y));
+    const float2 c = __ldg(table + rope_table_index(i, k, half));
+    const uint32_t oa = (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3) + 2 * (ea & 7);
+    const uint32_t ob = (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3) + 2 * (eb & 7);
+    for (int s = 0; s < 2; ++s) {
+      uint8_t* tile = s ? q1 : q0;
+      uint16_t* pa = reinterpret_cast<uint16_t*>(tile + oa);
+      uint16_t* pb = reinterpret_cast<uint16_t*>(tile + ob);
+      const float x = __uint_as_float((uint32_t)*pa << 16), y = __uint_as_float((uint32_t)*pb << 16);
+      *pa = __bfloat16_as_ushort(__float2bfloat16_rn(x * c.x - y * c.y));
+      *pb = __bfloat16_as_ushort(__float2bfloat16_rn(y * c.x + x * c.y));
+    }
   }
 }
 
@@ -197,14 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.q_full[s], 1);
-      mbar_init(&sm.q_ready[s], BM);
       mbar_init(&sm.q_empty[s], 1);
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_free[s], BM);
-      mbar_init(&sm.p_full[s], BM);
       mbar_init(&sm.alpha_full[s], BM);
       mbar_init(&sm.alpha_empty[s], BM);
-      mbar_init(&sm.o_ready[s], BM);
       mbar_init(&sm.pv_done[s], 1);
       mbar_init(&sm.l_full[s], BM);
       mbar_init(&sm.l_empty[s], BM);
@@ -219,6 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
     }
+    mbar_init(&sm.q_ready, BM);
+    mbar_init(&sm.s_free, 2 * BM);
+    mbar_init(&sm.pv_ready, 4 * BM);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -267,9 +294,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_4d(&q_map, 64, h, M.i0, M.b);
           }
           if (a.rotary_dim > 0) {
+            // the tile's positions are whole groups of 32 (i0 % 128 == 0)
             const int half = a.rotary_dim / 2;
-            const uint32_t bytes = (uint32_t)(min(BM, a.S - M.i0) * half * sizeof(float2)) & ~15u;
-            if (bytes > 0) bulk_prefetch_l2(a.table + (size_t)M.i0 * half, bytes);
+            const uint32_t bytes = (uint32_t)(((min(BM, a.S - M.i0) + 31) >> 5) * rope_table_couples(half) * 512);
+            bulk_prefetch_l2(a.table + rope_table_index(M.i0, 0, half), bytes);
           }
         }
         return true;
@@ -345,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
         const int n_kv = decode_tile(a, t).n_kv;
-        if (!mbar_wait(&sm.q_ready[0], it & 1, abort_flag) || !mbar_wait(&sm.q_ready[1], it & 1, abort_flag)) {
+        if (!mbar_wait(&sm.q_ready, it & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 3);
           ok = false;
           break;
@@ -353,8 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = -1; j < n_kv && ok; ++j) {
           if (j + 1 < n_kv) {
             const int g1 = G + j + 1, ki = kc + j + 1;
-            ok = (g1 == 0 || (mbar_wait(&sm.s_free[0], (g1 - 1) & 1, abort_flag) &&
-                              mbar_wait(&sm.s_free[1], (g1 - 1) & 1, abort_flag))) &&
+            ok = (g1 == 0 || mbar_wait(&sm.s_free, (g1 - 1) & 1, abort_flag)) &&
                  mbar_wait(&sm.k_full[ki % NK], (ki / NK) & 1, abort_flag);
             if (!ok) {
               fail(abort_flag, kErrPrefill + 4);
@@ -378,8 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (j >= 0) {
             const int g = G + j, vi = vc + j;
-            ok = mbar_wait(&sm.p_full[0], g & 1, abort_flag) && mbar_wait(&sm.o_ready[0], g & 1, abort_flag) &&
-                 mbar_wait(&sm.p_full[1], g & 1, abort_flag) && mbar_wait(&sm.o_ready[1], g & 1, abort_flag) &&
+            ok = mbar_wait(&sm.pv_ready, g & 1, abort_flag) &&
                  mbar_wait(&sm.v_full[vi % NV], (vi / NV) & 1, abort_flag);
             if (!ok) {
               fail(abort_flag, kErrPrefill + 5);
@@ -447,32 +473,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile(a, t);
       const int i = T.i0 + row;
-      // ---- Q rotation of this slot's tile (rows beyond S stay zero); the
-      // table row is fetched before the tile's arrival is awaited
-      const int half = a.rotary_dim / 2;
-      const bool rot = a.rotary_dim > 0 && i < a.S;
-      const bool vec = (half & 7) == 0;
-      float4 tb[32];
-      {
-        // rows without rotation read row 0; entries past half/2 repeat the last one
-        const float4* cs4 = reinterpret_cast<const float4*>(a.table + (size_t)(rot && vec ? i : 0) * half);
-        const int last = (rot && vec) ? half / 2 - 1 : 0;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) tb[k] = (rot && vec) ? __ldg(cs4 + min(k, last)) : make_float4(1.f, 0.f, 1.f, 0.f);
-      }
-      if (!warp_wait(&sm.q_full[s], it & 1, abort_flag)) {
-        fail(abort_flag, kErrPrefill + 6);
-        break;
-      }
-      if (rot) {
-        if (vec)
-          rotate_q_row_vec(sm.q[s], row, half, tb);
-        else
-          rotate_q_row_scalar(sm.q[s], row, half, a.table + (size_t)i * half);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&sm.q_ready[s]);
-
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < T.n_kv; ++j) {
         const int key0 = (T.kt_lo + j) * BN;
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&sm.s_free[s]);  // S_s may be overwritten by the next QK^T
+        mbar_arrive(&sm.s_free);  // S_s may be overwritten by the next QK^T
         // which mask bounds cut this key tile (uniform over the tile):
         // hi -- some key lies after some row (the diagonal tile);
         // lo -- some key lies at or before row - W (the band's first tile)
@@ -526,9 +526,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 128; e += 2) {
           const uint64_t y = f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), cc, mm);
-          float y0, y1;
-          f2_unpack(y, y0, y1);
-          const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+          float p0, p1;
+          if (poly_column_pair(e >> 1)) {
+            f2_unpack(exp2_poly2(y), p0, p1);
+          } else {
+            float y0, y1;
+            f2_unpack(y, y0, y1);
+            p0 = fast_exp2(y0);
+            p1 = fast_exp2(y1);
+          }
           sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(p0, p1));
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
@@ -547,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(sm.p[s] + (ch >> 3) * kBoxBytes + sw128_off(row, ch & 7)) =
               make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         fence_proxy_async_smem();
-        mbar_arrive(&sm.p_full[s]);
+        mbar_arrive(&sm.pv_ready);
         float s0, s1;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
         l = l * alpha + (s0 + s1);
@@ -567,8 +573,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsCorrection>();
     const int row = threadIdx.x & (BM - 1);
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    // RoPE of a tile's queries, both head slots, in shared memory (rows at
+    // or beyond S stay as loaded: zero)
+    auto prepare_q = [&](int t_q, int it_q) -> bool {
+      if (!warp_wait(&sm.q_full[0], it_q & 1, abort_flag) || !warp_wait(&sm.q_full[1], it_q & 1, abort_flag)) {
+        fail(abort_flag, kErrPrefill + 6);
+        return false;
+      }
+      const int i = decode_tile(a, t_q).i0 + row;
+      if (a.rotary_dim > 0 && i < a.S) {
+        const int half = a.rotary_dim / 2;
+        if ((half & 7) == 0)
+          rotate_q_rows_vec(sm.q[0], sm.q[1], row, half,
+                            reinterpret_cast<const float4*>(a.table) +
+                                ((((size_t)(i >> 5) * rope_table_couples(half)) << 5) + (i & 31)));
+        else
+          rotate_q_rows_scalar(sm.q[0], sm.q[1], row, i, half, a.table);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.q_ready);
+      return true;
+    };
     int it = 0, G = 0;
-    bool ok = true;
+    bool ok = blockIdx.x >= (unsigned)n_tiles || prepare_q(blockIdx.x, 0);
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile(a, t);
       const int i = T.i0 + row;
@@ -609,10 +636,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           tc_fence_before();
-          mbar_arrive(&sm.o_ready[s]);
+          mbar_arrive(&sm.pv_ready);
         }
       }
       if (!ok) break;
+      // the next tile's QK^T waits only for its rotated Q: prepare it before
+      // this tile's epilogue
+      if (t + (int)gridDim.x < n_tiles && !prepare_q(t + gridDim.x, it + 1)) {
+        ok = false;
+        break;
+      }
       // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged in p[s] for
       // the store warp (P_s(last) is consumed once that slot's P.V is done)
       for (int s = 0; s < 2 && ok; ++s) {

@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(256) rope_kernel(const RopeArgs a) {
   }
   if (a.table && active && b == 0 && blockIdx.y == 0) {
     for (int e = 0; e < 8; ++e)
-      if (L.role[e] == 1) a.table[(long long)s_idx * (r / 2) + L.freq[e]] = make_float2(c[e], s[e]);
+      if (L.role[e] == 1) a.table[rope_table_index(s_idx, L.freq[e], r / 2)] = make_float2(c[e], s[e]);
   }
 
   const int hs = blockIdx.y, nhs = gridDim.y;

@@ -22,6 +22,21 @@ enum : int {
 
 // ------------------------------------------------------------------ RoPE
 
+// Cos/sin table of the prefill: one float2 (cos, sin) per (position i, rotary
+// pair k < r/2), stored so that 32 consecutive positions read the same two
+// pairs from 512 contiguous bytes: groups of 32 positions, within a group the
+// couples of pairs (k/2) in order, within a couple the 32 positions, within a
+// position the two pairs.  A warp whose lanes hold 32 consecutive query rows
+// then loads a 16-byte (two-pair) slice per lane fully coalesced.
+__host__ __device__ __forceinline__ int rope_table_couples(int half) { return (half + 1) >> 1; }
+__host__ __device__ __forceinline__ long long rope_table_index(long long i, int k, int half) {
+  return ((((i >> 5) * rope_table_couples(half) + (k >> 1)) << 5) + (i & 31)) * 2 + (k & 1);
+}
+// bytes for positions 0..S-1 (whole groups of 32)
+__host__ __device__ __forceinline__ long long rope_table_bytes(long long S, int half) {
+  return ((S + 31) >> 5) * rope_table_couples(half) * 32 * 16;
+}
+
 struct RopeArgs {
   int B, S, Hq, Hkv;
   int rotary_dim;            // even, 0..128
@@ -35,7 +50,7 @@ struct RopeArgs {
   uint16_t* v_cache;
   int cache_capacity;        // C
   int window;                // W >= 1 or -1 (slot rule)
-  float2* table;             // [S][rotary_dim/2] (cos, sin) of positions 0..S-1, or nullptr
+  float2* table;             // cos/sin of positions 0..S-1 (rope_table_index layout), or nullptr
   int rotate;                // 0: theta == 0 or rotary_dim == 0 (copies only)
   double inv_freq[kMaxRotaryHalf];
 };
@@ -49,7 +64,7 @@ struct PrefillArgs {
   int window;                // W >= 1 or -1
   int rotary_dim;            // rotary dims applied to Q in-kernel (0: none)
   float scale_log2;          // softmax_scale * log2(e)
-  const float2* table;       // [S][rotary_dim/2] cos/sin, when rotary_dim > 0
+  const float2* table;       // cos/sin (rope_table_index layout), when rotary_dim > 0
   const float* gate;         // [B,S,Hq] or nullptr
   int n_q_tiles;             // ceil(S / 128)
   int n_head_pairs;          // ceil(G / 2)

@@ -64,6 +64,11 @@ def test_workspace_sizes(lib):
     k_bytes = 8192 * 8 * 128 * 2
     table = 8192 * 64 * 8
     assert ws == k_bytes + table
+    # the table holds whole groups of 32 positions and whole couples of pairs:
+    # S = 100 -> 4 groups, r = 6 -> 3 pairs -> 2 couples of 32 x 16 bytes
+    odd = api.LayerParams(4, 2, 128, -1, 1e4, 6)
+    k_odd = (1 * 100 * 2 * 128 * 2 + 255) // 256 * 256
+    assert api.prefill_workspace_size(odd, 1, 100) == k_odd + 4 * 2 * 512
     assert api.prefill_workspace_size(api.LayerParams(32, 2, 128, -1, 0.0, 128), 4, 16384) == 0
     # sliding decode: one split, no workspace; full decode: split-K partials
     assert api.decode_workspace_size(p, 64, 131072) == 0

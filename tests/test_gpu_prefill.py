@@ -49,7 +49,8 @@ def test_ragged_lengths(cuda_device, S, W):
     check_no_device_error()
 
 
-@pytest.mark.parametrize("theta,r", [(5e6, 64), (0.0, 128), (5e5, 32), (1e4, 6), (1e4, 0)])
+@pytest.mark.parametrize("theta,r", [(5e6, 64), (0.0, 128), (5e5, 32), (1e4, 16), (1e4, 24), (1e4, 6), (1e4, 2),
+                                     (1e4, 0)])
 def test_rope_variants(cuda_device, theta, r):
     p = api.LayerParams(8, 2, 128, 200, theta, r)
     _check_all_rows(cuda_device, p, 1, 384, seed=300 + r)
