@@ -67,8 +67,8 @@ constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
 // setmaxnreg split of the 128 x 512 registers the CTA is launched with
 constexpr uint32_t kRegsLaunch = 128;
-constexpr uint32_t kRegsSoftmax = 184;
-constexpr uint32_t kRegsCorrection = 88;
+constexpr uint32_t kRegsSoftmax = 176;
+constexpr uint32_t kRegsCorrection = 104;
 constexpr uint32_t kRegsOther = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
@@ -158,32 +158,54 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 // memory (two 64-dim boxes each, 128-byte swizzle): pairs (k, k + r/2) for
 // k < r/2.  Vector form for 16 | r: per 8-dim chunk, four 16-byte table
 // slices (two pairs each) that the warp's 32 rows load from 512 contiguous
-// bytes apiece.
+// bytes apiece.  The slices of the first kRopeAhead chunks are loaded by
+// rope_table_preload (before the tile's arrival is awaited); each chunk's
+// registers are refilled with the slices of the chunk kRopeAhead ahead as
+// soon as it is done, so several loads are always in flight.
+constexpr int kRopeAhead = 3;  // chunks whose table slices are in flight
+
+struct RopeSlices {
+  float4 t[kRopeAhead][4];
+};
+
+__device__ __forceinline__ void rope_table_preload(RopeSlices& r, const float4* __restrict__ tgroup, int n_chunks) {
+#pragma unroll
+  for (int c = 0; c < kRopeAhead; ++c)
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      if (c < n_chunks) r.t[c][w] = __ldg(tgroup + (size_t)(c * 4 + w) * 32);
+}
+
 __device__ __forceinline__ void rotate_q_rows_vec(uint8_t* q0, uint8_t* q1, int row, int half,
-                                                  const float4* __restrict__ tgroup) {
-#pragma unroll 1
-  for (int c0 = 0; c0 < half / 8; ++c0) {
-    const int ea = c0 * 8, eb = ea + half;
-    float4 t[4];
+                                                  const float4* __restrict__ tgroup, RopeSlices& r) {
+  const int n_chunks = half / 8;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) t[w] = __ldg(tgroup + (size_t)(c0 * 4 + w) * 32);  // pairs ea+2w, ea+2w+1
-    const uint32_t oa = (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3);
-    const uint32_t ob = (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3);
+  for (int c0 = 0; c0 < 8; ++c0) {
+    if (c0 < n_chunks) {
+      const int ea = c0 * 8, eb = ea + half;
+      const uint32_t oa = (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3);
+      const uint32_t ob = (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3);
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      uint8_t* tile = s ? q1 : q0;
-      uint4 A = *reinterpret_cast<uint4*>(tile + oa), Bv = *reinterpret_cast<uint4*>(tile + ob);
-      uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
-      uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
+      for (int s = 0; s < 2; ++s) {
+        uint8_t* tile = s ? q1 : q0;
+        uint4 A = *reinterpret_cast<uint4*>(tile + oa), Bv = *reinterpret_cast<uint4*>(tile + ob);
+        uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
+        uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
-        const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
-        a32[w] = pack_bf16x2(x0 * t[w].x - y0 * t[w].y, x1 * t[w].z - y1 * t[w].w);
-        b32[w] = pack_bf16x2(y0 * t[w].x + x0 * t[w].y, y1 * t[w].z + x1 * t[w].w);
+        for (int w = 0; w < 4; ++w) {
+          const float4 t = r.t[c0 % kRopeAhead][w];  // (cos, sin) of pairs ea+2w and ea+2w+1
+          const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
+          const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
+          a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
+          b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
+        }
+        *reinterpret_cast<uint4*>(tile + oa) = A;
+        *reinterpret_cast<uint4*>(tile + ob) = Bv;
       }
-      *reinterpret_cast<uint4*>(tile + oa) = A;
-      *reinterpret_cast<uint4*>(tile + ob) = Bv;
+      if (c0 + kRopeAhead < n_chunks) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) r.t[c0 % kRopeAhead][w] = __ldg(tgroup + (size_t)((c0 + kRopeAhead) * 4 + w) * 32);
+      }
     }
   }
 }
@@ -492,20 +514,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.s_free);  // S_s may be overwritten by the next QK^T
         // which mask bounds cut this key tile (uniform over the tile):
         // hi -- some key lies after some row (the diagonal tile);
-        // lo -- some key lies at or before row - W (the band's first tile)
+        // lo -- some key lies at or before row - W (the band's first tile).
+        // On a cut tile each 32-column chunk is, for the warp's 32 rows,
+        // either wholly masked (skipped: P = 0), wholly visible, or compared
+        // column by column.
         const bool cut_hi = key0 + BN - 1 > T.i0;
         const bool cut_lo = a.window > 0 && key0 < T.i0 + BM - a.window;
+        uint32_t masked = 0;  // bit q: chunk q masked for every row of the warp
         if (cut_hi || cut_lo) {
           const int hi = cut_hi ? i - key0 : BN;                     // columns > hi are masked
           const int lo = cut_lo ? i - a.window + 1 - key0 : -1;      // columns < lo are masked
 #pragma unroll
-          for (int e = 0; e < 128; ++e)
-            if (e > hi || e < lo) v[e] = __float_as_uint(-INFINITY);
+          for (int q = 0; q < 4; ++q) {
+            const int c0 = 32 * q;
+            if (__all_sync(0xffffffffu, hi < c0 || lo > c0 + 31)) {
+              masked |= 1u << q;
+            } else if (!__all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31)) {
+#pragma unroll
+              for (int e = c0; e < c0 + 32; ++e)
+                if (e > hi || e < lo) v[e] = __float_as_uint(-INFINITY);
+            }
+          }
         }
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 128; e += 2)
-          mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        for (int q = 0; q < 4; ++q) {
+          if (!((masked >> q) & 1u)) {
+#pragma unroll
+            for (int e = 32 * q; e < 32 * q + 32; e += 2)
+              mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+          }
+        }
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
         const float m_use = (mt - m > kRescaleThreshold) ? mt : m;  // m = -inf: always take mt
         const float m_safe = m_use == -INFINITY ? 0.f : m_use;
@@ -524,19 +563,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[64];
 #pragma unroll
-        for (int e = 0; e < 128; e += 2) {
-          const uint64_t y = f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), cc, mm);
-          float p0, p1;
-          if (poly_column_pair(e >> 1)) {
-            f2_unpack(exp2_poly2(y), p0, p1);
+        for (int q = 0; q < 4; ++q) {
+          if ((masked >> q) & 1u) {
+#pragma unroll
+            for (int e = 32 * q; e < 32 * q + 32; e += 2) pk[e >> 1] = 0u;
           } else {
-            float y0, y1;
-            f2_unpack(y, y0, y1);
-            p0 = fast_exp2(y0);
-            p1 = fast_exp2(y1);
+#pragma unroll
+            for (int e = 32 * q; e < 32 * q + 32; e += 2) {
+              const uint64_t y = f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), cc, mm);
+              float p0, p1;
+              if (poly_column_pair(e >> 1)) {
+                f2_unpack(exp2_poly2(y), p0, p1);
+              } else {
+                float y0, y1;
+                f2_unpack(y, y0, y1);
+                p0 = fast_exp2(y0);
+                p1 = fast_exp2(y1);
+              }
+              sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(p0, p1));
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
           }
-          sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(p0, p1));
-          pk[e >> 1] = pack_bf16x2(p0, p1);
         }
         // p[s] is free once P_s(j-1).V has completed; at a tile's first key
         // tile it holds the previous tile's output until the store has read
@@ -576,17 +623,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // RoPE of a tile's queries, both head slots, in shared memory (rows at
     // or beyond S stay as loaded: zero)
     auto prepare_q = [&](int t_q, int it_q) -> bool {
+      const int i = decode_tile(a, t_q).i0 + row;
+      const int half = a.rotary_dim / 2;
+      const bool rot = a.rotary_dim > 0 && i < a.S;
+      const bool vec = (half & 7) == 0;
+      const float4* tgroup =
+          reinterpret_cast<const float4*>(a.table) + ((((size_t)(i >> 5) * rope_table_couples(half)) << 5) + (i & 31));
+      RopeSlices slices;
+      if (rot && vec) rope_table_preload(slices, tgroup, half / 8);
       if (!warp_wait(&sm.q_full[0], it_q & 1, abort_flag) || !warp_wait(&sm.q_full[1], it_q & 1, abort_flag)) {
         fail(abort_flag, kErrPrefill + 6);
         return false;
       }
-      const int i = decode_tile(a, t_q).i0 + row;
-      if (a.rotary_dim > 0 && i < a.S) {
-        const int half = a.rotary_dim / 2;
-        if ((half & 7) == 0)
-          rotate_q_rows_vec(sm.q[0], sm.q[1], row, half,
-                            reinterpret_cast<const float4*>(a.table) +
-                                ((((size_t)(i >> 5) * rope_table_couples(half)) << 5) + (i & 31)));
+      if (rot) {
+        if (vec)
+          rotate_q_rows_vec(sm.q[0], sm.q[1], row, half, tgroup, slices);
         else
           rotate_q_rows_scalar(sm.q[0], sm.q[1], row, i, half, a.table);
       }
