@@ -19,11 +19,10 @@
 // output store of neighbouring tiles overlap with the tensor-core work.
 //
 // Warp roles (16 warps, registers rebalanced with setmaxnreg):
-//   warps 0-3   head slot 0: softmax (thread = query row)
+//   warps 0-3   head slot 0: Q rotation, softmax (thread = query row)
 //   warps 4-7   head slot 1: same
-//   warps 8-11  O rescaling ("correction"), the RoPE of the next tile's Q
-//               (both slots) and the epilogue (O/l * gate -> bf16 -> the
-//               slot's P buffer in shared memory)
+//   warps 8-11  O rescaling ("correction") and the epilogue (O/l * gate ->
+//               bf16 -> the slot's P buffer in shared memory)
 //   warp 12     tcgen05.mma issuer (one thread)
 //   warp 13     TMA producer (one thread)
 //   warp 14     TMA store of the output tiles (one thread)
@@ -83,7 +82,7 @@ struct PrefillSmem {
   float alpha[2][BM];
   float lsum[2][BM];
   uint64_t q_full[2], q_empty[2];
-  uint64_t q_ready;  // both slots' Q rotated (128 arrivals)
+  uint64_t q_ready;  // both slots' Q rotated (256 arrivals)
   uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
   uint64_t s_full[2], alpha_full[2], alpha_empty[2], pv_done[2];
   uint64_t s_free;    // both slots have read S (256 arrivals)
@@ -154,78 +153,55 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// Rotate query row `row` (position i) of both head slots' Q tiles in shared
-// memory (two 64-dim boxes each, 128-byte swizzle): pairs (k, k + r/2) for
-// k < r/2.  Vector form for 16 | r: per 8-dim chunk, four 16-byte table
-// slices (two pairs each) that the warp's 32 rows load from 512 contiguous
-// bytes apiece.  The slices of the first kRopeAhead chunks are loaded by
-// rope_table_preload (before the tile's arrival is awaited); each chunk's
-// registers are refilled with the slices of the chunk kRopeAhead ahead as
-// soon as it is done, so several loads are always in flight.
-constexpr int kRopeAhead = 3;  // chunks whose table slices are in flight
-
-struct RopeSlices {
-  float4 t[kRopeAhead][4];
-};
-
-__device__ __forceinline__ void rope_table_preload(RopeSlices& r, const float4* __restrict__ tgroup, int n_chunks) {
+// Rotate query row `row` (position i) of a Q tile in shared memory (two
+// 64-dim boxes, 128-byte swizzle): pairs (k, k + r/2) for k < r/2.  Vector
+// form for 16 | r: tb holds the row's 16-byte table slices (two pairs each),
+// loaded before the tile's arrival is awaited; the warp's 32 rows load each
+// slice index from 512 contiguous bytes.
+__device__ __forceinline__ void rope_table_load(float4 (&tb)[32], const float4* __restrict__ tgroup, int half) {
+  // slices past half/2 repeat the last one: unconditional loads stay in registers
+  const int last = half / 2 - 1;
 #pragma unroll
-  for (int c = 0; c < kRopeAhead; ++c)
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-      if (c < n_chunks) r.t[c][w] = __ldg(tgroup + (size_t)(c * 4 + w) * 32);
+  for (int k = 0; k < 32; ++k) tb[k] = __ldg(tgroup + (size_t)min(k, last) * 32);
 }
 
-__device__ __forceinline__ void rotate_q_rows_vec(uint8_t* q0, uint8_t* q1, int row, int half,
-                                                  const float4* __restrict__ tgroup, RopeSlices& r) {
-  const int n_chunks = half / 8;
+__device__ __forceinline__ void rotate_q_row_vec(uint8_t* tile, int row, int half, const float4 (&tb)[32]) {
 #pragma unroll
   for (int c0 = 0; c0 < 8; ++c0) {
-    if (c0 < n_chunks) {
+    if (c0 * 8 < half) {
       const int ea = c0 * 8, eb = ea + half;
-      const uint32_t oa = (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3);
-      const uint32_t ob = (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3);
+      uint4* pa = reinterpret_cast<uint4*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3));
+      uint4* pb = reinterpret_cast<uint4*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3));
+      uint4 A = *pa, Bv = *pb;
+      uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
+      uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        uint8_t* tile = s ? q1 : q0;
-        uint4 A = *reinterpret_cast<uint4*>(tile + oa), Bv = *reinterpret_cast<uint4*>(tile + ob);
-        uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
-        uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float4 t = r.t[c0 % kRopeAhead][w];  // (cos, sin) of pairs ea+2w and ea+2w+1
-          const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
-          const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
-          a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
-          b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
-        }
-        *reinterpret_cast<uint4*>(tile + oa) = A;
-        *reinterpret_cast<uint4*>(tile + ob) = Bv;
+      for (int w = 0; w < 4; ++w) {
+        const float4 t = tb[c0 * 4 + w];  // (cos, sin) of pairs ea+2w and ea+2w+1
+        const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
+        const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
+        a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
+        b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
       }
-      if (c0 + kRopeAhead < n_chunks) {
-#pragma unroll
-        for (int w = 0; w < 4; ++w) r.t[c0 % kRopeAhead][w] = __ldg(tgroup + (size_t)((c0 + kRopeAhead) * 4 + w) * 32);
-      }
+      *pa = A;
+      *pb = Bv;
     }
   }
 }
 
 // Element-wise form for any even r.
-__device__ __forceinline__ void rotate_q_rows_scalar(uint8_t* q0, uint8_t* q1, int row, int i, int half,
-                                                     const float2* __restrict__ table) {
+__device__ __forceinline__ void rotate_q_row_scalar(uint8_t* tile, int row, int i, int half,
+                                                    const float2* __restrict__ table) {
   for (int k = 0; k < half; ++k) {
     const int ea = k, eb = k + half;
     const float2 c = __ldg(table + rope_table_index(i, k, half));
     const uint32_t oa = (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3) + 2 * (ea & 7);
     const uint32_t ob = (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3) + 2 * (eb & 7);
-    for (int s = 0; s < 2; ++s) {
-      uint8_t* tile = s ? q1 : q0;
-      uint16_t* pa = reinterpret_cast<uint16_t*>(tile + oa);
-      uint16_t* pb = reinterpret_cast<uint16_t*>(tile + ob);
-      const float x = __uint_as_float((uint32_t)*pa << 16), y = __uint_as_float((uint32_t)*pb << 16);
-      *pa = __bfloat16_as_ushort(__float2bfloat16_rn(x * c.x - y * c.y));
-      *pb = __bfloat16_as_ushort(__float2bfloat16_rn(y * c.x + x * c.y));
-    }
+    uint16_t* pa = reinterpret_cast<uint16_t*>(tile + oa);
+    uint16_t* pb = reinterpret_cast<uint16_t*>(tile + ob);
+    const float x = __uint_as_float((uint32_t)*pa << 16), y = __uint_as_float((uint32_t)*pb << 16);
+    *pa = __bfloat16_as_ushort(__float2bfloat16_rn(x * c.x - y * c.y));
+    *pb = __bfloat16_as_ushort(__float2bfloat16_rn(y * c.x + x * c.y));
   }
 }
 
@@ -265,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
     }
-    mbar_init(&sm.q_ready, BM);
+    mbar_init(&sm.q_ready, 2 * BM);
     mbar_init(&sm.s_free, 2 * BM);
     mbar_init(&sm.pv_ready, 4 * BM);
     mbar_init(&sm.drain, 1);
@@ -495,6 +471,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile(a, t);
       const int i = T.i0 + row;
+      // ---- RoPE of this slot's Q tile (rows at or beyond S stay as loaded:
+      // zero); the first table slices are requested before Q is awaited
+      {
+        const int half = a.rotary_dim / 2;
+        const bool rot = a.rotary_dim > 0 && i < a.S;
+        const bool vec = (half & 7) == 0;
+        const float4* tgroup = reinterpret_cast<const float4*>(a.table) +
+                               ((((size_t)(i >> 5) * rope_table_couples(half)) << 5) + (i & 31));
+        float4 tb[32];
+        if (rot && vec) {
+          rope_table_load(tb, tgroup, half);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) tb[k] = make_float4(1.f, 0.f, 1.f, 0.f);
+        }
+        if (!warp_wait(&sm.q_full[s], it & 1, abort_flag)) {
+          fail(abort_flag, kErrPrefill + 6);
+          break;
+        }
+        if (rot) {
+          if (vec)
+            rotate_q_row_vec(sm.q[s], row, half, tb);
+          else
+            rotate_q_row_scalar(sm.q[s], row, i, half, a.table);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.q_ready);
+      }
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < T.n_kv; ++j) {
         const int key0 = (T.kt_lo + j) * BN;
@@ -620,33 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsCorrection>();
     const int row = threadIdx.x & (BM - 1);
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    // RoPE of a tile's queries, both head slots, in shared memory (rows at
-    // or beyond S stay as loaded: zero)
-    auto prepare_q = [&](int t_q, int it_q) -> bool {
-      const int i = decode_tile(a, t_q).i0 + row;
-      const int half = a.rotary_dim / 2;
-      const bool rot = a.rotary_dim > 0 && i < a.S;
-      const bool vec = (half & 7) == 0;
-      const float4* tgroup =
-          reinterpret_cast<const float4*>(a.table) + ((((size_t)(i >> 5) * rope_table_couples(half)) << 5) + (i & 31));
-      RopeSlices slices;
-      if (rot && vec) rope_table_preload(slices, tgroup, half / 8);
-      if (!warp_wait(&sm.q_full[0], it_q & 1, abort_flag) || !warp_wait(&sm.q_full[1], it_q & 1, abort_flag)) {
-        fail(abort_flag, kErrPrefill + 6);
-        return false;
-      }
-      if (rot) {
-        if (vec)
-          rotate_q_rows_vec(sm.q[0], sm.q[1], row, half, tgroup, slices);
-        else
-          rotate_q_rows_scalar(sm.q[0], sm.q[1], row, i, half, a.table);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&sm.q_ready);
-      return true;
-    };
     int it = 0, G = 0;
-    bool ok = blockIdx.x >= (unsigned)n_tiles || prepare_q(blockIdx.x, 0);
+    bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile(a, t);
       const int i = T.i0 + row;
@@ -691,12 +670,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      // the next tile's QK^T waits only for its rotated Q: prepare it before
-      // this tile's epilogue
-      if (t + (int)gridDim.x < n_tiles && !prepare_q(t + gridDim.x, it + 1)) {
-        ok = false;
-        break;
-      }
       // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged in p[s] for
       // the store warp (P_s(last) is consumed once that slot's P.V is done)
       for (int s = 0; s < 2 && ok; ++s) {
