@@ -71,6 +71,27 @@ def decode_bytes(c, lens) -> int:
     return keys * c.Hkv * 128 * 2 * 2 + c.B * c.Hq * (128 * 2 * 2 + 4)
 
 
+# DRAM traffic per launch of the prefill attention kernel from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/prefill_kernel_step37_sliding.md).
+# It describes only the kernel source it was taken on, so it is reported only
+# while csrc/prefill.cuh still hashes to the recorded digest, else null.
+PREFILL_TRAFFIC = {
+    "workload": "step37_sliding_B1_S8192_Hq96_Hkv8_W512",
+    "bytes": 404.2e6,
+    "source_sha256": "54e6d9e2edc9cb68d56387909b30d94b2216d904e9100f9621e4b6d5175439a1",
+}
+
+
+def measured_prefill_traffic(workload: str):
+    import hashlib
+    path = os.path.join(ROOT, "full_gqa_attention_swa_b200", "csrc", "prefill.cuh")
+    with open(path, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if workload == PREFILL_TRAFFIC["workload"] and digest == PREFILL_TRAFFIC["source_sha256"]:
+        return PREFILL_TRAFFIC["bytes"]
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -382,7 +403,7 @@ def main():
             "data": "synthetic N(0,1) bf16 q/k/v, N(0,1) fp32 gate logits (seeded)", "config": cfg,
             "clocks": clocks, "gpu_launches": launches}
     line["roofline"] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                        "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                        "frac": achieved / peaks["bf16_tflops"], "traffic": measured_prefill_traffic(c.name),
                         "peak_source": f"{peak_src} bf16 burst",
                         "kernel": "swa_attn_prefill (key-RoPE pre-pass + attention kernel), CUDA events"}
     if rank == 0 and not args.no_e2e:
