@@ -101,6 +101,16 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time: every rank takes part (same collective, same
+    order) and every rank gets the maximum."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def combine_ranks(elapsed_ms_per_rank, n_gpus: int, units_per_rank: float):
     """Whole-job throughput: units of all ranks over the slowest rank's time."""
     t = max(elapsed_ms_per_rank)
@@ -376,22 +386,25 @@ def main():
 
     if args.only.startswith("decode"):
         dc = configs.DECODE_SLIDING if args.only == "decode_sliding" else configs.DECODE_FULL
+        if dist is not None:
+            dist.barrier()
         d_ms, nbytes = bench_decode(dc, max(args.steps, 1), max(args.warmup, 3), dev)
-        gbs = nbytes / (d_ms / 1e3) / 1e9
+        d_ms = max_over_ranks(d_ms, dist, dev)
+        gbs = nbytes * world / (d_ms / 1e3) / 1e9
         if rank == 0:
             print(json.dumps({"metric": "decode HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": world,
                               "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": d_ms,
                               "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
                               "config": {"workload": dc.name},
                               "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                           "frac": gbs / peaks["hbm_gbs"], "traffic": None}}), flush=True)
+                                           "frac": gbs / world / peaks["hbm_gbs"], "traffic": None}}), flush=True)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
         return
 
     ms, clocks, launches = bench_prefill(c, args.steps, max(args.warmup, 3), dev, dist)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
     value, _ = combine_ranks([ms], world, flops * args.steps / 1e12)   # TFLOP/s over all ranks
     per_step_ms = ms / args.steps
     achieved = flops / (per_step_ms / 1e3) / 1e12
