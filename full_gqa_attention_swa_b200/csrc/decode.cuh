@@ -11,9 +11,11 @@
 //
 // Work split: one CTA per (sequence b, kv-head, split of `chunk` keys).  The
 // CTA serves all G q-heads of its kv-head, so each cache byte is read once.
-// A producer warp streams 64-key K and V blocks into shared memory with TMA
-// (128-byte swizzle, multi-stage mbarrier ring); four consumer warps each take
-// 16 keys of every block.  The G (<= 16) query rows are the M dimension of
+// A producer warp streams 32-key K and V blocks into shared memory with TMA
+// (128-byte swizzle, three-stage mbarrier ring); two consumer warps each take
+// 16 keys of every block.  At 48 KB of stages a CTA, four CTAs share an SM,
+// so a batch of up to 592 (sequence, kv-head, split) CTAs runs in one wave
+// with 192 KB of cache reads in flight per SM.  The G (<= 16) query rows are the M dimension of
 // m16n8k16 bf16 MMAs (fp32 accumulate): S = Q K^T, an online softmax over the
 // fragment rows with quad shuffles, then O += P V with P re-packed from the S
 // fragments.  The bound is HBM bandwidth: 512 cache bytes per key against
@@ -26,12 +28,14 @@ namespace swa {
 namespace decode_detail {
 
 constexpr int KB = kDecodeKeyBlock;        // keys per stage
-constexpr int kConsumerWarps = 4;
-constexpr int kKeysPerWarp = KB / kConsumerWarps;   // 16
+constexpr int kKeysPerWarp = 16;                    // the k16 of one P.V MMA
+constexpr int kConsumerWarps = KB / kKeysPerWarp;   // 2
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr uint32_t kBoxBytes = KB * 128;   // 64 keys x 64 dims x 2 B
-constexpr uint32_t kStageBytes = 4 * kBoxBytes;  // K lo/hi + V lo/hi = 32 KB
+constexpr int kCtasPerSm = 4;
+constexpr uint32_t kBoxBytes = KB * 128;   // 32 keys x 64 dims x 2 B
+constexpr uint32_t kStageBytes = 4 * kBoxBytes;  // K lo/hi + V lo/hi = 16 KB
 constexpr int kMergeStride = kHeadDim + 8;       // floats per merged row (padding vs bank conflicts)
+static_assert(KB % kKeysPerWarp == 0 && kBoxBytes % 1024 == 0, "stage boxes must stay 1024-byte aligned");
 
 template <int NS>
 struct DecodeSmem {
@@ -73,7 +77,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
 __device__ __forceinline__ float sigmoidf_(float g) { return 1.f / (1.f + __expf(-g)); }
 
 template <int NS>
-__global__ void __launch_bounds__(kThreads) decode_split_kernel(const DecodeArgs a,
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_split_kernel(const DecodeArgs a,
                                                                 const __grid_constant__ CUtensorMap k_map,
                                                                 const __grid_constant__ CUtensorMap v_map) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -260,8 +264,10 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const DecodeArgs
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
     named_bar_sync(1, kConsumerWarps * 32);  // every warp is done reading the stages
+    static_assert(sizeof(float) * kConsumerWarps * 16 * kMergeStride <= sizeof(sm.stage),
+                  "the merge reuses the stages");
     if (!*abort_flag) {
-      float* mo = reinterpret_cast<float*>(sm.stage[0]);  // [warps][16][kMergeStride]
+      float* mo = reinterpret_cast<float*>(sm.stage[0]);  // [warps][16][kMergeStride], over the idle stages
       float* mine = mo + warp * 16 * kMergeStride;
 #pragma unroll
       for (int n = 0; n < 16; ++n) {
@@ -279,26 +285,31 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const DecodeArgs
     named_bar_sync(1, kConsumerWarps * 32);
     if (!*abort_flag) {
       const float* mo = reinterpret_cast<const float*>(sm.stage[0]);
-      const int d = threadIdx.x;  // 0..127: one head dim per thread
+      // each consumer thread merges two adjacent head dims of every row
+      const int d = 2 * threadIdx.x;
+      static_assert(2 * 32 * kConsumerWarps == kHeadDim, "two dims per consumer thread");
       for (int r = 0; r < G; ++r) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.m_part[w][r]);
-        float lsum = 0.f, acc = 0.f;
+        float lsum = 0.f, acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
           const float f = sm.m_part[w][r] == -INFINITY ? 0.f : fast_exp2(sm.m_part[w][r] - M);
           lsum += f * sm.l_part[w][r];
-          acc += f * mo[(w * 16 + r) * kMergeStride + d];
+          const float2 v = *reinterpret_cast<const float2*>(mo + (w * 16 + r) * kMergeStride + d);
+          acc0 += f * v.x;
+          acc1 += f * v.y;
         }
         const int h = kvh * G + r;
         if (a.max_splits == 1) {
           const float gt = a.gate ? sigmoidf_(a.gate[(size_t)b * a.Hq + h]) : 1.f;
-          const float y = acc / lsum * gt;
-          a.out[((size_t)b * a.Hq + h) * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+          const float sc = gt / lsum;
+          *reinterpret_cast<uint32_t*>(a.out + ((size_t)b * a.Hq + h) * kHeadDim + d) =
+              pack_bf16x2(acc0 * sc, acc1 * sc);
         } else {
           const size_t slot = ((size_t)b * a.Hq + h) * a.max_splits + split;
-          a.part_o[slot * kHeadDim + d] = acc;
+          *reinterpret_cast<float2*>(a.part_o + slot * kHeadDim + d) = make_float2(acc0, acc1);
           if (d == 0) a.part_ml[slot] = make_float2(M, lsum);
         }
       }

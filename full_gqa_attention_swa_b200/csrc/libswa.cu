@@ -154,11 +154,16 @@ DecodePlan plan_decode(const swa_layer_params* p, int B, int max_len) {
   DecodePlan pl{};
   const long long kb = swa::kDecodeKeyBlock;
   const long long n_vis = p->window > 0 ? (max_len < p->window ? max_len : p->window) : max_len;
-  // aim for about three resident CTAs per SM over the whole batch
-  long long c = ((long long)B * p->num_kv_heads * n_vis + 148 * 3 - 1) / (148 * 3);
+  // aim for about four resident CTAs per SM (the decode kernel's occupancy)
+  // over the whole batch; when the (sequence, kv-head) pairs alone fill at
+  // least half of those slots and a whole sequence fits one chunk, splitting
+  // would only add waves (and the combine)
+  const long long slots = 148 * 4, items = (long long)B * p->num_kv_heads;
+  long long c = (items * n_vis + slots - 1) / slots;
   c = (c + kb - 1) / kb * kb;
   if (c < 256) c = 256;
   if (c > 4096) c = 4096;
+  if (2 * items >= slots && n_vis <= 4096) c = n_vis;
   if (c >= n_vis) {
     pl.chunk = (int)((n_vis + kb - 1) / kb * kb);
     pl.splits = 1;

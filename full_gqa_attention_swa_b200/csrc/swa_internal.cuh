@@ -96,6 +96,6 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& k_map, const CUtensorMap& v_map,
                           cudaStream_t stream);
 
-constexpr int kDecodeKeyBlock = 64;   // keys per pipeline stage
+constexpr int kDecodeKeyBlock = 32;   // keys per pipeline stage
 
 }  // namespace swa
