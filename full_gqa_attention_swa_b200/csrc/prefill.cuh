@@ -26,21 +26,22 @@
 //   warp 12     tcgen05.mma issuer (one thread)
 //   warp 13     TMA producer (one thread)
 //   warp 14     TMA store of the output tiles (one thread)
-//   warp 15     idle
+//   warp 15     folds K / V arrivals into the issuer's barriers (one thread)
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384)
 // O1 [384,512).  P (bf16) goes to a shared-memory buffer per head slot.
 //
 // Per key tile j and head slot s:
-//   MMA:     S_s = Q_s K_j^T            -> s_full[s]
+//   MMA:     S_s = Q_s K_j^T            -> s_full (both slots)
 //   softmax: read S_s                   -> s_free (both slots: S(j+1) may start)
 //            m, alpha                   -> alpha_full[s]
 //            P_s = 2^(S_s - m) -> smem  -> pv_ready
 //   correct: wait PV_s(j-1), O_s *= alpha (skipped when alpha == 1 for the
 //            whole warp)                -> pv_ready
-//   MMA:     O_s += P_s V_j             -> pv_done[s] (also frees p[s])
+//   MMA:     O_s += P_s V_j             -> pv_done (both slots; frees the P buffers)
 // The MMA thread waits on one barrier per hand-off (s_free, pv_ready) rather
 // than one per slot and producer: each wait is a shared-memory round trip that
-// queues behind the softmax warps' SFU traffic on the same sub-partition.
+// queues behind the softmax warps' SFU traffic on the same sub-partition.  A
+// helper thread folds the K / V tile arrivals into those two barriers.
 // The exponentials run on the SFU (a polynomial path on the FMA pipe exists,
 // see poly_column_pair).
 // The max used for the exponentials only moves when the new row max exceeds
@@ -84,9 +85,11 @@ struct PrefillSmem {
   uint64_t q_full[2], q_empty[2];
   uint64_t q_ready;  // both slots' Q rotated (256 arrivals)
   uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
-  uint64_t s_full[2], alpha_full[2], alpha_empty[2], pv_done[2];
-  uint64_t s_free;    // both slots have read S (256 arrivals)
-  uint64_t pv_ready;  // both slots' P written and O rescaled (512 arrivals)
+  uint64_t alpha_full[2], alpha_empty[2];
+  uint64_t s_full;    // S of both slots complete
+  uint64_t pv_done;   // P.V of both slots complete (frees both P buffers)
+  uint64_t s_free;    // both slots have read S, and the next K tile has landed (256 + 1 arrivals)
+  uint64_t pv_ready;  // both slots' P written and O rescaled, and the V tile has landed (512 + 1)
   uint64_t l_full[2], l_empty[2];
   uint64_t ost_full[2];  // output tile staged in p[s]
   uint64_t pfree[2];     // the store of that tile has read p[s]
@@ -224,10 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.q_full[s], 1);
       mbar_init(&sm.q_empty[s], 1);
-      mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.alpha_full[s], BM);
       mbar_init(&sm.alpha_empty[s], BM);
-      mbar_init(&sm.pv_done[s], 1);
       mbar_init(&sm.l_full[s], BM);
       mbar_init(&sm.l_empty[s], BM);
       mbar_init(&sm.ost_full[s], BM);
@@ -242,8 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_empty[i], 1);
     }
     mbar_init(&sm.q_ready, 2 * BM);
-    mbar_init(&sm.s_free, 2 * BM);
-    mbar_init(&sm.pv_ready, 4 * BM);
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.pv_done, 1);
+    mbar_init(&sm.s_free, 2 * BM + 1);
+    mbar_init(&sm.pv_ready, 4 * BM + 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -379,8 +382,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = -1; j < n_kv && ok; ++j) {
           if (j + 1 < n_kv) {
             const int g1 = G + j + 1, ki = kc + j + 1;
-            ok = (g1 == 0 || mbar_wait(&sm.s_free, (g1 - 1) & 1, abort_flag)) &&
-                 mbar_wait(&sm.k_full[ki % NK], (ki / NK) & 1, abort_flag);
+            // s_free(g1 - 1) includes the arrival of K(g1); only the very
+            // first K tile is awaited here
+            ok = g1 == 0 ? mbar_wait(&sm.k_full[0], 0, abort_flag) : mbar_wait(&sm.s_free, (g1 - 1) & 1, abort_flag);
             if (!ok) {
               fail(abort_flag, kErrPrefill + 4);
               break;
@@ -393,8 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_ss(tmem, qd0 + off, kd + off, idesc_qk, kk > 0);
               umma_ss(tmem + 128, qd1 + off, kd + off, idesc_qk, kk > 0);
             }
-            umma_commit(&sm.s_full[0]);
-            umma_commit(&sm.s_full[1]);
+            umma_commit(&sm.s_full);
             umma_commit(&sm.k_empty[ki % NK]);
             if (j + 2 == n_kv) {
               umma_commit(&sm.q_empty[0]);
@@ -403,8 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (j >= 0) {
             const int g = G + j, vi = vc + j;
-            ok = mbar_wait(&sm.pv_ready, g & 1, abort_flag) &&
-                 mbar_wait(&sm.v_full[vi % NV], (vi / NV) & 1, abort_flag);
+            ok = mbar_wait(&sm.pv_ready, g & 1, abort_flag);  // includes the arrival of V(g)
             if (!ok) {
               fail(abort_flag, kErrPrefill + 5);
               break;
@@ -419,8 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_ss(tmem + 256, pd0 + aoff, vd + boff, idesc_pv, acc);
               umma_ss(tmem + 384, pd1 + aoff, vd + boff, idesc_pv, acc);
             }
-            umma_commit(&sm.pv_done[0]);
-            umma_commit(&sm.pv_done[1]);
+            umma_commit(&sm.pv_done);
             umma_commit(&sm.v_empty[vi % NV]);
           }
         }
@@ -431,6 +432,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // all MMAs issued by this thread complete before the CTA moves on
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, 200000000ull);
+    } else if (warp == 15 && lane == 0) {
+      // ========================================================== arrivals
+      // Folds the landing of each K / V tile into the barrier the MMA thread
+      // waits on anyway: s_free(g - 1) counts the arrival of K(g), pv_ready(g)
+      // that of V(g), in the issuer's order.  Before arriving for a phase it
+      // waits for the previous phase to complete, so an early arrival never
+      // counts toward the wrong phase.
+      int G = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int n_kv = decode_tile(a, t).n_kv;
+        for (int j = -1; j < n_kv && ok; ++j) {
+          const int g1 = G + j + 1;
+          if (j + 1 < n_kv && g1 >= 1) {
+            ok = (g1 < 2 || mbar_wait(&sm.s_free, (g1 - 2) & 1, abort_flag)) &&
+                 mbar_wait(&sm.k_full[g1 % NK], (g1 / NK) & 1, abort_flag);
+            if (ok) mbar_arrive(&sm.s_free);
+          }
+          if (ok && j >= 0) {
+            const int g = G + j;
+            ok = (g < 1 || mbar_wait(&sm.pv_ready, (g - 1) & 1, abort_flag)) &&
+                 mbar_wait(&sm.v_full[g % NV], (g / NV) & 1, abort_flag);
+            if (ok) mbar_arrive(&sm.pv_ready);
+          }
+        }
+        G += n_kv;
+      }
+      if (!ok) fail(abort_flag, kErrPrefill + 18);
     } else if (warp == 14 && lane == 0) {
       // ========================================================== output store
       // The epilogue stages each slot's output tile in that slot's P buffer;
@@ -502,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < T.n_kv; ++j) {
         const int key0 = (T.kt_lo + j) * BN;
-        if (!warp_wait(&sm.s_full[s], (G + j) & 1, abort_flag)) {
+        if (!warp_wait(&sm.s_full, (G + j) & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 7);
           ok = false;
           break;
@@ -593,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tile it holds the previous tile's output until the store has read
         // it.  (S(j) completing implies P(j-2).V completed, since its commit
         // covers every earlier MMA, so these waits are never two phases ahead.)
-        if (j > 0 ? !warp_wait(&sm.pv_done[s], (G + j - 1) & 1, abort_flag)
+        if (j > 0 ? !warp_wait(&sm.pv_done, (G + j - 1) & 1, abort_flag)
                   : (it > 0 && !warp_wait(&sm.pfree[s], (it - 1) & 1, abort_flag))) {
           fail(abort_flag, kErrPrefill + 16);
           ok = false;
@@ -645,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float alpha = sm.alpha[s][row];
           mbar_arrive(&sm.alpha_empty[s]);
           if (j > 0) {
-            if (!warp_wait(&sm.pv_done[s], (G + j - 1) & 1, abort_flag)) {
+            if (!warp_wait(&sm.pv_done, (G + j - 1) & 1, abort_flag)) {
               fail(abort_flag, kErrPrefill + 10);
               ok = false;
               break;
@@ -673,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged in p[s] for
       // the store warp (P_s(last) is consumed once that slot's P.V is done)
       for (int s = 0; s < 2 && ok; ++s) {
-        if (!warp_wait(&sm.pv_done[s], (G + T.n_kv - 1) & 1, abort_flag) ||
+        if (!warp_wait(&sm.pv_done, (G + T.n_kv - 1) & 1, abort_flag) ||
             !warp_wait(&sm.l_full[s], it & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 11);
           ok = false;

@@ -35,8 +35,9 @@ def test_tiny_config_all_rows(cuda_device):
 
 
 @pytest.mark.parametrize("W", [1, 2, 63, 64, 65, 127, 128, 129, 300, -1])
-def test_window_sweep(cuda_device, W):
-    p = api.LayerParams(4, 2, 128, W, 1e4, 128)
+@pytest.mark.parametrize("Hq", [4, 8])  # G = 2: single-SM kernel; G = 4: CTA-pair kernel
+def test_window_sweep(cuda_device, W, Hq):
+    p = api.LayerParams(Hq, 2, 128, W, 1e4, 128)
     _check_all_rows(cuda_device, p, 1, 300, seed=100 + max(W, 0))
     check_no_device_error()
 
@@ -57,7 +58,7 @@ def test_rope_variants(cuda_device, theta, r):
     check_no_device_error()
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(6, 2), (2, 2), (3, 1), (16, 1)])
+@pytest.mark.parametrize("Hq,Hkv", [(6, 2), (2, 2), (3, 1), (16, 1), (8, 1), (12, 1)])
 def test_gqa_groups(cuda_device, Hq, Hkv):
     p = api.LayerParams(Hq, Hkv, 128, 100, 1e4, 128)
     _check_all_rows(cuda_device, p, 3, 200, seed=400 + Hq)
@@ -120,4 +121,22 @@ def test_full_size_sampled_rows(cuda_device, cfg):
     ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy(), rows=rows)
     got = out.cpu()[torch.from_numpy(rows[:, 0]), torch.from_numpy(rows[:, 1]), torch.from_numpy(rows[:, 2])]
     assert_close(got, ref, cfg.name)
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("Hq,Hkv,W,B", [(16, 2, 512, 4), (16, 2, -1, 4), (4, 2, 300, 8), (12, 1, 200, 8)],
+                         ids=["pair-sliding", "pair-causal", "single-sliding", "pair-G12"])
+def test_persistent_multi_tile(cuda_device, Hq, Hkv, W, B):
+    """More work tiles than CTAs (or CTA pairs): every CTA runs several tiles
+    back to back, so tile boundaries inside one persistent CTA are checked."""
+    S, seed = 2048, 700 + Hq + B
+    p = api.LayerParams(Hq, Hkv, 128, W, 1e4, 128)
+    d = inputs.prefill_inputs(B, S, Hq, Hkv, 128, seed)
+    dev = {k: t.to(cuda_device) for k, t in d.items()}
+    out = api.attn_prefill(p, dev["q"], dev["k"], dev["v"], dev["gate"])
+    torch.cuda.synchronize()
+    rows = prefill_rows_sample(B, S, Hq, W, seed, n_random=160)
+    ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy(), rows=rows)
+    got = out.cpu()[torch.from_numpy(rows[:, 0]), torch.from_numpy(rows[:, 1]), torch.from_numpy(rows[:, 2])]
+    assert_close(got, ref, f"multi-tile Hq{Hq} Hkv{Hkv} W{W} B{B}")
     check_no_device_error()
