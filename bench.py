@@ -51,6 +51,15 @@ def visible_pairs(S: int, window: int) -> int:
     return W * (W + 1) // 2 + (S - W) * W
 
 
+def chunk_visible_pairs(pos0: int, S: int, window: int) -> int:
+    """Visible (i, j) pairs of query rows pos0 .. pos0 + S - 1."""
+    return visible_pairs(pos0 + S, window) - visible_pairs(pos0, window)
+
+
+def chunk_flops(c) -> float:
+    return 4.0 * 128 * c.Hq * c.B * chunk_visible_pairs(c.pos0, c.S, c.window)
+
+
 def prefill_flops(c) -> float:
     """Unmasked FLOPs: QK^T and P.V over visible pairs, 2 * 2 * D each."""
     return 4.0 * 128 * c.Hq * c.B * visible_pairs(c.S, c.window)
@@ -222,6 +231,48 @@ def bench_prefill(c, steps: int, warmup: int, dev, dist=None):
     return ms, clocks.summary(), launches
 
 
+def bench_prefill_chunk(c, steps: int, warmup: int, dev):
+    """Continued prefill: each step runs swa_attn_prefill_chunk on the same
+    chunk against a cache holding positions < pos0 (synthetic N(0,1) keys
+    and values); the chunk re-appends itself each step.  Two input sets
+    rotate (the full layer's cache of 134 MB alone exceeds L2)."""
+    from full_gqa_attention_swa_b200 import api
+
+    p = api.LayerParams(c.Hq, c.Hkv, 128, c.window, c.theta, c.rotary_dim)
+    C = c.window if c.window > 0 else c.pos0 + c.S
+    sets = []
+    for r in range(2):
+        d = inputs.prefill_inputs(c.B, c.S, c.Hq, c.Hkv, 128, c.seed + 31 * r, device=dev)
+        cache = inputs.decode_inputs(c.B, c.Hq, c.Hkv, 128, C, c.seed + 31 * r + 7, device=dev)
+        d["k_cache"], d["v_cache"] = cache["k_cache"], cache["v_cache"]
+        sets.append(d)
+    out = torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(api.prefill_chunk_workspace_size(p, c.B, c.S, c.pos0), 1), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        d = sets[i % 2]
+        api.attn_prefill_chunk(p, c.pos0, d["q"], d["k"], d["v"], d["gate"], d["k_cache"], d["v_cache"], out=out,
+                               workspace=ws, stream=stream)
+
+    for i in range(max(warmup, 3)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / steps
+    assert api.device_error() == 0, "a kernel reported a bounded-wait timeout"
+    del sets
+    torch.cuda.empty_cache()
+    return ms
+
+
 def bench_prefill_e2e(c, steps: int, dev):
     """Same metric through the public API with host buffers: pinned host
     inputs copied in and the output copied back every step."""
@@ -331,7 +382,8 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--workload", default=configs.STEP_SLIDING.name, choices=sorted(configs.PREFILL))
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode_sliding", "decode_full"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode_sliding", "decode_full", "chunk_sliding",
+                                       "chunk_full"], default="all",
                     help="run one leg only (profiling); prints that leg's own JSON line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
@@ -384,6 +436,24 @@ def main():
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
 
+    if args.only.startswith("chunk"):
+        cc = configs.CHUNK_SLIDING if args.only == "chunk_sliding" else configs.CHUNK_FULL
+        c_ms = bench_prefill_chunk(cc, max(args.steps, 1), max(args.warmup, 3), dev)
+        c_ms = max_over_ranks(c_ms, dist, dev)
+        tf = chunk_flops(cc) * world / (c_ms / 1e3) / 1e12
+        if rank == 0:
+            print(json.dumps({"metric": "continued prefill unmasked TFLOP/s", "value": tf, "unit": "TFLOP/s",
+                              "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+                              "ms_per_step": c_ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                              "config": {"workload": cc.name},
+                              "roofline": {"bound": "tensor", "achieved": tf / world, "peak": peaks["bf16_tflops"],
+                                           "unit": "TFLOP/s", "frac": tf / world / peaks["bf16_tflops"],
+                                           "traffic": None}}), flush=True)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
     if args.only.startswith("decode"):
         dc = configs.DECODE_SLIDING if args.only == "decode_sliding" else configs.DECODE_FULL
         if dist is not None:
@@ -434,6 +504,13 @@ def main():
                 extra[dc.name] = {"ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                                   "peak_source": f"{peak_src} hbm copy"}
             line["decode"] = extra
+            chunks = {}
+            for cc in (configs.CHUNK_SLIDING, configs.CHUNK_FULL):
+                c_ms = bench_prefill_chunk(cc, 20 if cc.window > 0 else 5, 3, dev)
+                tf = chunk_flops(cc) / (c_ms / 1e3) / 1e12
+                chunks[cc.name] = {"ms": c_ms, "TFLOP/s": tf, "frac_bf16": tf / peaks["bf16_tflops"],
+                                   "peak_source": f"{peak_src} bf16 burst"}
+            line["prefill_chunk"] = chunks
         if args.cpu_budget > 0:
             r, n, dt, thr = oracle_sample_rate(c, args.cpu_budget)
             line["cpu_baseline"] = {"value": r, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",

@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "SWA_OK", 1: "SWA_ERR_INVALID_ARG", 2: "SWA_ERR_UNSUPPORTED",
 # every function include/swa.h declares
 SYMBOLS = ("swa_rope_qk", "swa_prefill_workspace_size", "swa_attn_prefill", "swa_decode_workspace_size",
            "swa_attn_decode", "swa_kv_cache_bytes", "swa_status_string", "swa_last_error_detail",
-           "swa_device_error", "swa_version", "swa_attn_decode_no_alloc")
+           "swa_device_error", "swa_version", "swa_attn_decode_no_alloc", "swa_prefill_chunk_workspace_size",
+           "swa_attn_prefill_chunk")
 
 # bytes of the static device array behind swa_attn_decode_no_alloc
 NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -103,6 +104,10 @@ def load(path: str = LIB_PATH):
     lib.swa_version.restype = ctypes.c_char_p
     lib.swa_attn_decode_no_alloc.argtypes = [P, i32, vp, vp, vp, vp, i32, vp, i32, vp, vp]
     lib.swa_attn_decode_no_alloc.restype = ctypes.c_int
+    lib.swa_prefill_chunk_workspace_size.argtypes = [P, i32, i32, i32]
+    lib.swa_prefill_chunk_workspace_size.restype = sz
+    lib.swa_attn_prefill_chunk.argtypes = [P, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+    lib.swa_attn_prefill_chunk.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -191,6 +196,38 @@ def attn_prefill(layer: LayerParams, q, k, v, gate=None, out=None, workspace=Non
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load().swa_attn_prefill(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(v), _ptr(gate),
                                    _ptr(out), _ptr(workspace), nbytes, _stream(stream)))
+    return out
+
+
+def prefill_chunk_workspace_size(layer: LayerParams, B: int, S: int, pos0: int) -> int:
+    return int(load().swa_prefill_chunk_workspace_size(ctypes.byref(layer.c()), B, S, pos0))
+
+
+def attn_prefill_chunk(layer: LayerParams, pos0: int, q, k, v, gate, k_cache, v_cache, out=None, workspace=None,
+                       stream=None):
+    """swa_attn_prefill_chunk: new tokens at positions pos0 .. pos0+S-1 (q
+    [B,S,Hq,D], k/v [B,S,Hkv,D] bf16, not rotated; gate [B,S,Hq] fp32 or None)
+    against the KV cache [B,Hkv,C,D] holding positions < pos0; appends the
+    chunk to the cache.  Returns out [B,S,Hq,D] bf16."""
+    B, S = q.shape[0], q.shape[1]
+    D = layer.head_dim
+    C = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (B, S, layer.num_q_heads, D))
+    _need(k, "k", torch.bfloat16, (B, S, layer.num_kv_heads, D))
+    _need(v, "v", torch.bfloat16, (B, S, layer.num_kv_heads, D))
+    _need(gate, "gate", torch.float32, (B, S, layer.num_q_heads))
+    _need(k_cache, "k_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, (B, S, layer.num_q_heads, D))
+    need = prefill_chunk_workspace_size(layer, B, S, pos0)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().swa_attn_prefill_chunk(ctypes.byref(layer.c()), B, S, int(pos0), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(gate), _ptr(k_cache), _ptr(v_cache), C, _ptr(out), _ptr(workspace),
+                                         nbytes, _stream(stream)))
     return out
 
 

@@ -47,6 +47,23 @@ class DecodeLayer:
     seed: int
 
 
+@dataclass(frozen=True)
+class ChunkLayer:
+    """A continued prefill: S new tokens at positions pos0 .. pos0 + S - 1
+    against a KV cache holding positions < pos0."""
+    name: str
+    B: int
+    pos0: int
+    S: int
+    Hq: int
+    Hkv: int
+    D: int
+    window: int
+    theta: float
+    rotary_dim: int
+    seed: int
+
+
 # tiny oracle case: B1 S256 Hq8 Hkv1 W64, theta 1e4 on all 128 dims
 TINY = PrefillLayer("tiny_B1_S256_Hq8_Hkv1_W64", 1, 256, 8, 1, 128, 64, 1e4, 128, 1000)
 
@@ -70,5 +87,13 @@ DECODE_SLIDING = DecodeLayer("decode_sliding_B64_Hq96_Hkv8_W512", 64, 96, 8, 128
 DECODE_FULL = DecodeLayer("decode_full_B64_Hq64_Hkv8", 64, 64, 8, 128, WINDOW_FULL, 5e6, 64,
                           4096, 131072, 131072, 1004)
 
+# continued prefill: the second half of the Step sliding and full prefills,
+# chunked against the cache the first half left
+CHUNK_SLIDING = ChunkLayer("step37_sliding_chunk_B1_pos4096_S4096_Hq96_Hkv8_W512", 1, 4096, 4096, 96, 8, 128,
+                           512, 1e4, 128, 1005)
+CHUNK_FULL = ChunkLayer("step37_full_chunk_B1_pos16384_S16384_Hq64_Hkv8", 1, 16384, 16384, 64, 8, 128,
+                        WINDOW_FULL, 5e6, 64, 1006)
+
 PREFILL = {c.name: c for c in (TINY, STEP_SLIDING, STEP_FULL, MUSE_SLIDING, MUSE_FULL)}
+CHUNK = {c.name: c for c in (CHUNK_SLIDING, CHUNK_FULL)}
 DECODE = {c.name: c for c in (DECODE_SLIDING, DECODE_FULL)}

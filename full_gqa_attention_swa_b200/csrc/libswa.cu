@@ -13,6 +13,7 @@
 #include "swa_internal.cuh"
 
 #include "decode.cuh"
+#include "kv_gather.cuh"
 #include "prefill.cuh"
 #include "rope.cuh"
 
@@ -114,6 +115,15 @@ swa_status encode_bshd(CUtensorMap* map, const void* base, int B, int S, int H, 
   return encode_bf16(map, base, 4, dims, strides, box);
 }
 
+// [B*Hkv, C, D] bf16 cache -> 3-D map {D, keys, B*Hkv} over the first `keys`
+// slots (later slots read as zero), box {64, rows, 1}.
+swa_status encode_cache_keys(CUtensorMap* map, const void* base, int BH, int C, int keys, int rows) {
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)keys, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)C * kHeadDim * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  return encode_bf16(map, base, 3, dims, strides, box);
+}
+
 // [B*Hkv, C, D] bf16 cache -> 3-D map {D, C, B*Hkv}, box {64, rows, 1}.
 swa_status encode_cache(CUtensorMap* map, const void* base, int BH, int C, int rows) {
   const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)C, (cuuint64_t)BH};
@@ -142,6 +152,33 @@ PrefillPlan plan_prefill(const swa_layer_params* p, int B, int S) {
     pl.table_bytes = round_up((size_t)swa::rope_table_bytes(S, p->rotary_dim / 2), 256);
   }
   pl.total = pl.k_bytes + pl.table_bytes;
+  return pl;
+}
+
+// Continued prefill: on a ring (sliding) layer the keys / values the chunk
+// attends to are assembled in the workspace (h earlier tokens + the chunk);
+// on a full layer the chunk is appended to the linear cache first and the
+// attention reads the cache in place.
+struct ChunkPlan {
+  bool rotate, ring;
+  int h;  // history rows per sequence (ring)
+  size_t k_bytes, v_bytes, table_bytes, total;
+};
+
+ChunkPlan plan_prefill_chunk(const swa_layer_params* p, int B, int S, int pos0) {
+  ChunkPlan pl{};
+  pl.rotate = rotates(p);
+  pl.ring = p->window > 0;
+  const size_t row = (size_t)p->num_kv_heads * kHeadDim * 2;
+  if (pl.ring) {
+    pl.h = pos0 < p->window - 1 ? pos0 : p->window - 1;
+    pl.k_bytes = round_up((size_t)B * (pl.h + S) * row, 256);
+    pl.v_bytes = pl.k_bytes;
+  } else if (pl.rotate) {
+    pl.k_bytes = round_up((size_t)B * S * row, 256);
+  }
+  if (pl.rotate) pl.table_bytes = round_up((size_t)swa::rope_table_bytes(S, p->rotary_dim / 2), 256);
+  pl.total = pl.k_bytes + pl.v_bytes + pl.table_bytes;
   return pl;
 }
 
@@ -374,6 +411,98 @@ swa_status swa_attn_prefill(const swa_layer_params* p, int32_t B, int32_t S, con
   a.n_q_tiles = (int)n_q_tiles;
   a.n_head_pairs = (G + 1) / 2;
   st = cuda_status(swa::launch_prefill(a, qm, km, vm, om, s), "prefill launch");
+  return st == SWA_OK ? ok() : st;
+}
+
+size_t swa_prefill_chunk_workspace_size(const swa_layer_params* p, int32_t B, int32_t S, int32_t pos0) {
+  if (check_layer(p) != SWA_OK || B < 0 || S < 0 || pos0 < 0) return 0;
+  return plan_prefill_chunk(p, B, S, pos0).total;
+}
+
+swa_status swa_attn_prefill_chunk(const swa_layer_params* p, int32_t B, int32_t S, int32_t pos0, const uint16_t* q,
+                                  const uint16_t* k, const uint16_t* v, const float* gate, uint16_t* k_cache,
+                                  uint16_t* v_cache, int32_t cache_capacity, uint16_t* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  swa_status st = check_layer(p);
+  if (st != SWA_OK) return st;
+  if (B < 0 || S < 0 || pos0 < 0) return fail(SWA_ERR_INVALID_ARG, "B=%d S=%d pos0=%d must be >= 0", B, S, pos0);
+  if ((long long)pos0 + S > 0x7FFFFFFFll) return fail(SWA_ERR_INVALID_ARG, "pos0 + S must stay below 2^31");
+  if ((long long)B * S == 0) return ok();
+  if (!q || !k || !v || !out || !k_cache || !v_cache)
+    return fail(SWA_ERR_INVALID_ARG, "q, k, v, k_cache, v_cache and out must be non-NULL");
+  const void* ptrs[] = {q, k, v, out, gate, k_cache, v_cache, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(SWA_ERR_INVALID_ARG, "tensor pointer %p is not 16-byte aligned", ptr);
+  if (p->window > 0 ? cache_capacity != p->window : (long long)cache_capacity < (long long)pos0 + S)
+    return fail(SWA_ERR_INVALID_ARG, "cache_capacity %d: must equal W on a sliding layer, be >= pos0 + S on a full one",
+                cache_capacity);
+  const ChunkPlan pl = plan_prefill_chunk(p, B, S, pos0);
+  if (pl.total > 0) {
+    if (!workspace) return fail(SWA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", pl.total);
+    if (workspace_bytes < pl.total)
+      return fail(SWA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, pl.total);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(SWA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  const int Hq = p->num_q_heads, Hkv = p->num_kv_heads, G = Hq / Hkv;
+  const long long n_q_tiles = ((long long)S + 127) / 128;
+  if (n_q_tiles * ((G + 1) / 2) * Hkv * (long long)B > 0x7FFFFFFFll)
+    return fail(SWA_ERR_UNSUPPORTED, "grid too large");
+
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  uint16_t* k_seq = pl.k_bytes ? reinterpret_cast<uint16_t*>(ws) : nullptr;
+  uint16_t* v_seq = pl.v_bytes ? reinterpret_cast<uint16_t*>(ws + pl.k_bytes) : nullptr;
+  float2* table = pl.rotate ? reinterpret_cast<float2*>(ws + pl.k_bytes + pl.v_bytes) : nullptr;
+  if (pl.ring) {
+    // the chunk attends to up to W - 1 earlier tokens: copy them out of the
+    // ring before the chunk's own tokens overwrite their slots
+    swa::KvGatherArgs g{};
+    g.B = B; g.S = S; g.Hkv = Hkv; g.h = pl.h; g.pos0 = pos0; g.window = p->window; g.capacity = cache_capacity;
+    g.k_cache = k_cache; g.v_cache = v_cache; g.v = v; g.k_seq = k_seq; g.v_seq = v_seq;
+    st = cuda_status(swa::launch_kv_gather(g, s), "history gather launch");
+    if (st != SWA_OK) return st;
+  }
+  // the chunk's keys: rotated at their positions (into the assembled sequence
+  // on a ring layer, into scratch on a full one) and, with the values,
+  // appended to the cache; the cos/sin table of the chunk's positions
+  swa::RopeArgs r{};
+  r.B = B; r.S = S; r.Hq = Hq; r.Hkv = Hkv; r.rotary_dim = p->rotary_dim; r.pos0 = pos0; r.pos = nullptr;
+  r.q = nullptr; r.k_src = k; r.v = v;
+  if (pl.ring) {
+    r.k_dst = k_seq; r.dst_rows = pl.h + S; r.dst_row_off = pl.h;
+  } else {
+    r.k_dst = pl.rotate ? k_seq : const_cast<uint16_t*>(k);  // without rotation nothing is written to k
+  }
+  r.k_cache = k_cache; r.v_cache = v_cache; r.cache_capacity = cache_capacity; r.window = p->window;
+  r.table = table; r.rotate = pl.rotate ? 1 : 0;
+  if (pl.rotate) fill_inv_freq(p, r.inv_freq);
+  st = cuda_status(swa::launch_rope(r, s), "rope (chunk keys) launch");
+  if (st != SWA_OK) return st;
+
+  CUtensorMap qm, km, vm, om;
+  if ((st = encode_bshd(&qm, q, B, S, Hq, 128)) != SWA_OK) return st;
+  if ((st = encode_bshd(&om, out, B, S, Hq, 128)) != SWA_OK) return st;
+  swa::PrefillArgs a{};
+  if (pl.ring) {
+    if ((st = encode_bshd(&km, k_seq, B, pl.h + S, Hkv, 128)) != SWA_OK) return st;
+    if ((st = encode_bshd(&vm, v_seq, B, pl.h + S, Hkv, 128)) != SWA_OK) return st;
+    a.q_off = pl.h;
+  } else {
+    // keys 0 .. pos0 + S - 1 straight from the linear cache
+    if ((st = encode_cache_keys(&km, k_cache, B * Hkv, cache_capacity, pos0 + S, 128)) != SWA_OK) return st;
+    if ((st = encode_cache_keys(&vm, v_cache, B * Hkv, cache_capacity, pos0 + S, 128)) != SWA_OK) return st;
+    a.q_off = pos0;
+    a.kv_cache_layout = 1;
+  }
+  a.B = B; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.window = p->window;
+  a.rotary_dim = pl.rotate ? p->rotary_dim : 0;
+  a.scale_log2 = scale_log2(p);
+  a.table = table;
+  a.gate = gate;
+  a.n_q_tiles = (int)n_q_tiles;
+  a.n_head_pairs = (G + 1) / 2;
+  st = cuda_status(swa::launch_prefill(a, qm, km, vm, om, s), "prefill (chunk) launch");
   return st == SWA_OK ? ok() : st;
 }
 

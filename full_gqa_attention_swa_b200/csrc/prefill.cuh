@@ -10,7 +10,9 @@
 // 6bit" explainer's theta = 0 (no rotation) on full layers.
 //
 // Work unit ("tile"): 128 query rows x two q-heads of the same kv-head, so
-// every K/V tile in shared memory feeds two 128x128 score tiles.  A tile
+// every K/V tile in shared memory feeds two 128x128 score tiles.  Query row r
+// sits at key-space position i = q_off + r (q_off > 0 when a chunk of queries
+// continues a sequence whose earlier keys are in the K/V source).  A tile
 // loops over the key tiles of its band [i0 - W + 1, i0 + 127]; key tiles
 // wholly outside the band are never loaded, and the mask is evaluated only
 // on tiles the band edge or the diagonal cuts.  The grid is persistent (one
@@ -99,11 +101,21 @@ struct PrefillSmem {
 };
 
 struct Tile {
-  int qt, kvh, b, h0, h1, i0, kt_lo, n_kv;
+  int qt, kvh, b, h0, h1;
+  int r0;  // first query row of the tile (rows of q / out / gate / cos-sin table)
+  int i0;  // its key-space position, q_off + r0 (masks and key ranges)
+  int kt_lo, n_kv;
   bool store1;
 };
 
+// Launch modes: a whole prefill (queries at key positions 0..S-1, K / V as
+// [B, S, Hkv, D]), a chunk over an assembled K / V sequence (queries offset by
+// q_off), and a chunk over a KV cache [B * Hkv, C, D] read in place.
+enum PrefillMode : int { kWhole = 0, kChunkSeq = 1, kChunkCache = 2 };
+
+template <int kMode>
 __device__ __forceinline__ Tile decode_tile(const PrefillArgs& a, int t) {
+  const int q_off = kMode == kWhole ? 0 : a.q_off;
   Tile T;
   const int per_qt = a.n_head_pairs * a.Hkv * a.B;
   T.qt = a.n_q_tiles - 1 - t / per_qt;  // latest query rows (most keys) first
@@ -115,8 +127,9 @@ __device__ __forceinline__ Tile decode_tile(const PrefillArgs& a, int t) {
   T.h0 = T.kvh * a.G + 2 * hp;
   T.h1 = T.kvh * a.G + min(2 * hp + 1, a.G - 1);
   T.store1 = 2 * hp + 1 < a.G;
-  T.i0 = T.qt * BM;
-  const int row_last = min(T.i0 + BM - 1, a.S - 1);
+  T.r0 = T.qt * BM;
+  T.i0 = q_off + T.r0;
+  const int row_last = q_off + min(T.r0 + BM - 1, a.S - 1);
   const int key_lo = a.window > 0 ? max(0, T.i0 - a.window + 1) : 0;
   T.kt_lo = key_lo / BN;
   T.n_kv = row_last / BN - T.kt_lo + 1;
@@ -208,6 +221,9 @@ __device__ __forceinline__ void rotate_q_row_scalar(uint8_t* tile, int row, int 
   }
 }
 
+// kMode (PrefillMode) is a template parameter so that the whole prefill
+// carries neither the query offset nor a per-load layout branch.
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap q_map,
                    const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
@@ -277,28 +293,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       int q_last[2] = {-1, -1};
       bool ok = true;
       auto load_q = [&](int t_q, int it_q) -> bool {
-        const Tile N = decode_tile(a, t_q);
+        const Tile N = decode_tile<kMode>(a, t_q);
         for (int s = 0; s < 2; ++s) {
           if (it_q > 0 && !mbar_wait(&sm.q_empty[s], (it_q - 1) & 1, abort_flag)) return false;
           mbar_arrive_expect_tx(&sm.q_full[s], kTileBytes);
           const int h = s ? N.h1 : N.h0;
-          tma_load_4d(sm.q[s], &q_map, &sm.q_full[s], 0, h, N.i0, N.b);
-          tma_load_4d(sm.q[s] + kBoxBytes, &q_map, &sm.q_full[s], 64, h, N.i0, N.b);
+          tma_load_4d(sm.q[s], &q_map, &sm.q_full[s], 0, h, N.r0, N.b);
+          tma_load_4d(sm.q[s] + kBoxBytes, &q_map, &sm.q_full[s], 64, h, N.r0, N.b);
           q_last[s] = it_q;
         }
         // warm L2 for the Q tiles and cos/sin rows of the tile after it
         if (t_q + (int)gridDim.x < n_tiles) {
-          const Tile M = decode_tile(a, t_q + gridDim.x);
+          const Tile M = decode_tile<kMode>(a, t_q + gridDim.x);
           for (int s = 0; s < 2; ++s) {
             const int h = s ? M.h1 : M.h0;
-            tma_prefetch_4d(&q_map, 0, h, M.i0, M.b);
-            tma_prefetch_4d(&q_map, 64, h, M.i0, M.b);
+            tma_prefetch_4d(&q_map, 0, h, M.r0, M.b);
+            tma_prefetch_4d(&q_map, 64, h, M.r0, M.b);
           }
           if (a.rotary_dim > 0) {
-            // the tile's positions are whole groups of 32 (i0 % 128 == 0)
+            // the tile's rows are whole groups of 32 (r0 % 128 == 0)
             const int half = a.rotary_dim / 2;
-            const uint32_t bytes = (uint32_t)(((min(BM, a.S - M.i0) + 31) >> 5) * rope_table_couples(half) * 512);
-            bulk_prefetch_l2(a.table + rope_table_index(M.i0, 0, half), bytes);
+            const uint32_t bytes = (uint32_t)(((min(BM, a.S - M.r0) + 31) >> 5) * rope_table_couples(half) * 512);
+            bulk_prefetch_l2(a.table + rope_table_index(M.r0, 0, half), bytes);
           }
         }
         return true;
@@ -314,11 +330,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap* map = is_v ? &v_map : &k_map;
         const int key0 = (T.kt_lo + j) * BN;
         mbar_arrive_expect_tx(full, kTileBytes);
-        tma_load_4d(dst, map, full, 0, T.kvh, key0, T.b);
-        tma_load_4d(dst + kBoxBytes, map, full, 64, T.kvh, key0, T.b);
+        if constexpr (kMode == kChunkCache) {  // KV cache [B * Hkv, C, D]
+          tma_load_3d(dst, map, full, 0, key0, T.b * a.Hkv + T.kvh);
+          tma_load_3d(dst + kBoxBytes, map, full, 64, key0, T.b * a.Hkv + T.kvh);
+        } else {
+          tma_load_4d(dst, map, full, 0, T.kvh, key0, T.b);
+          tma_load_4d(dst + kBoxBytes, map, full, 64, T.kvh, key0, T.b);
+        }
         if (is_v) {
           v_end = idx + 1;
-          if (j + 1 < T.n_kv) {  // the next V comes through L2
+          if (kMode != kChunkCache && j + 1 < T.n_kv) {  // the next V comes through L2
             tma_prefetch_4d(&v_map, 0, T.kvh, key0 + BN, T.b);
             tma_prefetch_4d(&v_map, 64, T.kvh, key0 + BN, T.b);
           }
@@ -329,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       if (blockIdx.x < (unsigned)n_tiles && !load_q(blockIdx.x, 0)) ok = false;
       for (int t = blockIdx.x; t < n_tiles && ok && !*abort_flag; t += gridDim.x, ++it) {
-        const Tile T = decode_tile(a, t);
+        const Tile T = decode_tile<kMode>(a, t);
         const bool has_next = t + (int)gridDim.x < n_tiles;
         for (int j = -1; j < T.n_kv && ok; ++j) {
           if (j + 1 < T.n_kv) ok = load_kv(false, T, j + 1);
@@ -373,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, G = 0, kc = 0, vc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const int n_kv = decode_tile(a, t).n_kv;
+        const int n_kv = decode_tile<kMode>(a, t).n_kv;
         if (!mbar_wait(&sm.q_ready, it & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 3);
           ok = false;
@@ -442,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int G = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int n_kv = decode_tile(a, t).n_kv;
+        const int n_kv = decode_tile<kMode>(a, t).n_kv;
         for (int j = -1; j < n_kv && ok; ++j) {
           const int g1 = G + j + 1;
           if (j + 1 < n_kv && g1 >= 1) {
@@ -467,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&o_map);
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-        const Tile T = decode_tile(a, t);
+        const Tile T = decode_tile<kMode>(a, t);
         bool ok = true;
         for (int s = 0; s < 2; ++s) {
           if (!mbar_wait(&sm.ost_full[s], it & 1, abort_flag)) {
@@ -477,8 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (s == 0 || T.store1) {
             const int h = s ? T.h1 : T.h0;
-            tma_store_4d(&o_map, sm.p[s], 0, h, T.i0, T.b);
-            tma_store_4d(&o_map, sm.p[s] + kBoxBytes, 64, h, T.i0, T.b);
+            tma_store_4d(&o_map, sm.p[s], 0, h, T.r0, T.b);
+            tma_store_4d(&o_map, sm.p[s] + kBoxBytes, 64, h, T.r0, T.b);
             bulk_commit_group();
           }
           bulk_wait_group_read0();
@@ -498,16 +519,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0, G = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-      const Tile T = decode_tile(a, t);
-      const int i = T.i0 + row;
+      const Tile T = decode_tile<kMode>(a, t);
+      const int r = T.r0 + row;  // query row
+      const int i = T.i0 + row;  // its key-space position
       // ---- RoPE of this slot's Q tile (rows at or beyond S stay as loaded:
       // zero); the first table slices are requested before Q is awaited
       {
         const int half = a.rotary_dim / 2;
-        const bool rot = a.rotary_dim > 0 && i < a.S;
+        const bool rot = a.rotary_dim > 0 && r < a.S;
         const bool vec = (half & 7) == 0;
         const float4* tgroup = reinterpret_cast<const float4*>(a.table) +
-                               ((((size_t)(i >> 5) * rope_table_couples(half)) << 5) + (i & 31));
+                               ((((size_t)(r >> 5) * rope_table_couples(half)) << 5) + (r & 31));
         float4 tb[32];
         if (rot && vec) {
           rope_table_load(tb, tgroup, half);
@@ -523,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (vec)
             rotate_q_row_vec(sm.q[s], row, half, tb);
           else
-            rotate_q_row_scalar(sm.q[s], row, i, half, a.table);
+            rotate_q_row_scalar(sm.q[s], row, r, half, a.table);
         }
         fence_proxy_async_smem();
         mbar_arrive(&sm.q_ready);
@@ -656,13 +678,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0, G = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-      const Tile T = decode_tile(a, t);
-      const int i = T.i0 + row;
+      const Tile T = decode_tile<kMode>(a, t);
+      const int r = T.r0 + row;  // query row
       // gate logits of this row for both head slots, fetched early
       float glog[2] = {0.f, 0.f};
-      if (a.gate && i < a.S) {
-        glog[0] = __ldg(a.gate + ((size_t)T.b * a.S + i) * a.Hq + T.h0);
-        glog[1] = __ldg(a.gate + ((size_t)T.b * a.S + i) * a.Hq + T.h1);
+      if (a.gate && r < a.S) {
+        glog[0] = __ldg(a.gate + ((size_t)T.b * a.S + r) * a.Hq + T.h0);
+        glog[1] = __ldg(a.gate + ((size_t)T.b * a.S + r) * a.Hq + T.h1);
       }
       for (int j = 0; j < T.n_kv && ok; ++j) {
         for (int s = 0; s < 2; ++s) {
@@ -748,9 +770,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace prefill_detail
 
-cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                           const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream) {
-  using namespace prefill_detail;
+namespace prefill_detail {
+
+template <int kMode>
+cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
+                             const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream) {
   const long long n_tiles = (long long)a.n_q_tiles * a.n_head_pairs * a.Hkv * a.B;
   if (n_tiles == 0) return cudaSuccess;
   if (n_tiles > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
@@ -758,12 +782,13 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const
   static int n_sm = 0;
   static bool checked = false;
   if (!checked) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(prefill_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // setmaxnreg redistributes the registers the CTA was launched with: the
     // kernel must be launched with exactly kRegsLaunch per thread
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, prefill_kernel);
+    e = cudaFuncGetAttributes(&fa, prefill_kernel<kMode>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != (int)kRegsLaunch) return cudaErrorInvalidConfiguration;
     int dev = 0;
@@ -774,8 +799,18 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const
     checked = true;
   }
   const int grid = (int)(n_tiles < n_sm ? n_tiles : n_sm);
-  prefill_kernel<<<grid, kThreads, smem, stream>>>(a, q_map, k_map, v_map, o_map);
+  prefill_kernel<kMode><<<grid, kThreads, smem, stream>>>(a, q_map, k_map, v_map, o_map);
   return cudaGetLastError();
+}
+
+}  // namespace prefill_detail
+
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
+                           const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream) {
+  using namespace prefill_detail;
+  if (a.kv_cache_layout) return launch_prefill_t<kChunkCache>(a, q_map, k_map, v_map, o_map, stream);
+  if (a.q_off) return launch_prefill_t<kChunkSeq>(a, q_map, k_map, v_map, o_map, stream);
+  return launch_prefill_t<kWhole>(a, q_map, k_map, v_map, o_map, stream);
 }
 
 }  // namespace swa

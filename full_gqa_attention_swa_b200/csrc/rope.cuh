@@ -118,8 +118,9 @@ __device__ __forceinline__ void rope_cos_sin(double angle, float* c, float* s) {
 }
 
 // grid.x: ceil(B*S*16 / blockDim.x); grid.y: head split (heads h with
-// h % gridDim.y == blockIdx.y).
-__global__ void __launch_bounds__(256) rope_kernel(const RopeArgs a) {
+// h % gridDim.y == blockIdx.y).  Memory-bound: at least three 256-thread
+// blocks per SM keep enough loads in flight (the register cap costs no spill).
+__global__ void __launch_bounds__(256, 3) rope_kernel(const RopeArgs a) {
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int chunk = (int)(tid & (kChunks - 1));
   const long long tok = tid >> 4;
@@ -154,17 +155,24 @@ __global__ void __launch_bounds__(256) rope_kernel(const RopeArgs a) {
     }
   }
   if (a.k_src) {
-    const bool in_place = a.k_dst == a.k_src;
+    const long long dst_tok = (long long)b * (a.dst_rows > 0 ? a.dst_rows : a.S) + a.dst_row_off + s_idx;
+    const bool in_place = a.k_dst == a.k_src && dst_tok == tk;
     long long slot = 0;
     bool slot_ok = true;
     if (a.k_cache) {
       slot = a.window > 0 ? (long long)(p % a.window) : (long long)p;
       slot_ok = p >= 0 && slot < a.cache_capacity;
       if (active && !slot_ok && chunk == 0 && hs == 0) record_error(kErrRope + 1);
+      if (a.window > 0 && !a.pos) {
+        // consecutive positions pos0 .. pos0 + S - 1 on a ring: only the last
+        // W are kept, so no two tokens of the call write one slot (explicit
+        // positions are the caller's promise of distinct slots)
+        slot_ok = slot_ok && p > a.pos0 + a.S - 1 - a.window;
+      }
     }
     for (int h = hs; h < a.Hkv; h += nhs) {
       const uint16_t* src = a.k_src + (tk * a.Hkv + h) * kHeadDim;
-      uint16_t* dst = a.k_dst + (tk * a.Hkv + h) * kHeadDim;
+      uint16_t* dst = a.k_dst + (dst_tok * a.Hkv + h) * kHeadDim;
       if (r > 0 || !in_place) rotate_chunk(src, dst, chunk, L, c, s, active, in_place);
       if (a.k_cache && active && slot_ok) {
         // the rotated chunk: re-read from dst when it was written, else rotate here

@@ -44,12 +44,14 @@ struct RopeArgs {
   const int32_t* pos;        // [B,S] or nullptr (pos0 + s)
   uint16_t* q;               // [B,S,Hq,D] rotated in place, or nullptr
   const uint16_t* k_src;     // [B,S,Hkv,D] or nullptr
-  uint16_t* k_dst;           // [B,S,Hkv,D] rotated keys (may alias k_src); required with k_src
+  uint16_t* k_dst;           // rotated keys, [B, dst_rows, Hkv, D] from row dst_row_off (may alias k_src); required with k_src
+  int dst_rows;              // rows per sequence of k_dst (0: S)
+  int dst_row_off;           // row of k_dst that token 0 of a sequence goes to
   const uint16_t* v;         // [B,S,Hkv,D], for the cache append
   uint16_t* k_cache;         // [B,Hkv,C,D] or nullptr
   uint16_t* v_cache;
   int cache_capacity;        // C
-  int window;                // W >= 1 or -1 (slot rule)
+  int window;                // W >= 1 or -1 (slot rule; with pos == nullptr a ring keeps the call's last W positions)
   float2* table;             // cos/sin of positions 0..S-1 (rope_table_index layout), or nullptr
   int rotate;                // 0: theta == 0 or rotary_dim == 0 (copies only)
   double inv_freq[kMaxRotaryHalf];
@@ -68,12 +70,32 @@ struct PrefillArgs {
   const float* gate;         // [B,S,Hq] or nullptr
   int n_q_tiles;             // ceil(S / 128)
   int n_head_pairs;          // ceil(G / 2)
+  int q_off;                 // key-space position of query row 0 (keys 0 .. q_off + S - 1); 0 for a whole prefill
+  int kv_cache_layout;       // 0: k/v maps {D, Hkv, keys, B}; 1: a KV cache, maps {D, keys, B * Hkv}
 };
 
-// q_map / o_map: 4-D {D, Hq, S, B}; k_map / v_map: 4-D {D, Hkv, S, B};
-// boxes {64, 1, 128, 1}, 128-byte swizzle.
+// q_map / o_map: 4-D {D, Hq, S, B}; k_map / v_map: 4-D {D, Hkv, q_off + S, B}
+// (any strides: a KV cache [B, Hkv, C, D] is addressed in place); boxes
+// {64, 1, 128, 1}, 128-byte swizzle.  Query row r sits at key-space position
+// q_off + r; the cos/sin table and the gate are indexed by r.
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
                            const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream);
+
+// ------------------------------------------------------ continued prefill
+
+struct KvGatherArgs {
+  int B, S, Hkv;
+  int h;                     // history tokens gathered per sequence (<= W - 1)
+  int pos0;                  // position of the chunk's first token
+  int window, capacity;      // the ring: W == C slots
+  const uint16_t* k_cache;   // [B, Hkv, C, D]
+  const uint16_t* v_cache;
+  const uint16_t* v;         // [B, S, Hkv, D] the chunk's values
+  uint16_t* k_seq;           // [B, h + S, Hkv, D]: rows 0..h-1 written here
+  uint16_t* v_seq;           // [B, h + S, Hkv, D]: all rows written here
+};
+
+cudaError_t launch_kv_gather(const KvGatherArgs& a, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 

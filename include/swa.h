@@ -91,6 +91,11 @@ typedef struct swa_layer_params {
  *            NULL.  Token at position p goes to slot p mod W on a sliding
  *            layer (C must equal W) and to slot p on a full layer (p < C is
  *            the caller's promise; C >= 1).  k must be given with caches.
+ *            On a sliding layer with pos == NULL only the last W positions
+ *            pos0 + S - W .. pos0 + S - 1 are written, so no two tokens of one
+ *            call write the same slot; with explicit positions, no two tokens
+ *            of one sequence in a call may map to the same slot (caller's
+ *            promise).
  *   The angle is p * theta^(-2k/rotary_dim), evaluated in fp64; the
  *   rotation itself runs in fp32 and the result is rounded to bf16.
  *   With theta == 0 or rotary_dim == 0, q/k are left unchanged and the
@@ -128,6 +133,48 @@ SWA_API size_t swa_prefill_workspace_size(const swa_layer_params* params, int32_
 SWA_API swa_status swa_attn_prefill(const swa_layer_params* params, int32_t B, int32_t S, const uint16_t* q,
                             const uint16_t* k, const uint16_t* v, const float* gate, uint16_t* out,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * swa_prefill_chunk_workspace_size -- bytes of workspace
+ * swa_attn_prefill_chunk needs for (params, B, S, pos0): on a sliding layer
+ * the keys and values the chunk attends to (up to W - 1 earlier tokens plus
+ * the chunk) as [B, h + S, Hkv, D] bf16 each, h = min(pos0, W - 1); on a full
+ * layer the rotated chunk keys [B, S, Hkv, D]; plus the cos/sin table of
+ * positions pos0 .. pos0 + S - 1 when the layer rotates.  Each part 256-byte
+ * aligned.  Returns 0 for invalid parameters.
+ */
+SWA_API size_t swa_prefill_chunk_workspace_size(const swa_layer_params* params, int32_t B, int32_t S,
+                                                 int32_t pos0);
+
+/*
+ * swa_attn_prefill_chunk -- continue a prefill: S new tokens at positions
+ * pos0 .. pos0 + S - 1 of each of B sequences whose tokens 0 .. pos0 - 1 are
+ * already in the KV cache (rotated keys, raw values, as swa_rope_qk or an
+ * earlier chunk wrote them).  Each new token attends to its visible keys --
+ * cached and new -- exactly as in swa_attn_prefill over the whole sequence
+ * (the same rows of the same result), and the chunk's keys and values are
+ * then in the cache, so decode or the next chunk can follow.  pos0 = 0
+ * is a whole prefill that also fills the cache.  (Step explainer section 2.2:
+ * the sliding layers' cache keeps the last W tokens, the KV cache prefill
+ * the page mentions; sections 2.3 for RoPE and the gate.)
+ *
+ *   q, k, v  [B, S, Hq | Hkv, D] bf16 of the new tokens, NOT rotated
+ *   gate     [B, S, Hq] fp32 logits, or NULL
+ *   k_cache, v_cache  [B, Hkv, C, D] bf16, C = cache_capacity: a sliding
+ *            layer's ring (C must equal W; position p in slot p mod W) or a
+ *            full layer's linear cache (slot p; C >= pos0 + S).  Read for
+ *            positions < pos0, written for the new positions (on a ring only
+ *            the last W of them).
+ *   out      [B, S, Hq, D] bf16
+ *   workspace / workspace_bytes: at least swa_prefill_chunk_workspace_size()
+ *            bytes, 256-byte aligned; overwritten.
+ *   No tensor may overlap another.  Positions pos0 + S must stay below 2^31.
+ */
+SWA_API swa_status swa_attn_prefill_chunk(const swa_layer_params* params, int32_t B, int32_t S, int32_t pos0,
+                                          const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                          const float* gate, uint16_t* k_cache, uint16_t* v_cache,
+                                          int32_t cache_capacity, uint16_t* out, void* workspace,
+                                          size_t workspace_bytes, void* stream);
 
 /*
  * swa_decode_workspace_size -- bytes of workspace swa_attn_decode needs for a

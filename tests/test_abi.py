@@ -33,7 +33,7 @@ def _P(**kw):
 
 def test_exports_every_declared_symbol(lib):
     declared = _declared()
-    assert len(declared) == len(api.SYMBOLS) == 11
+    assert len(declared) == len(api.SYMBOLS) == 13
     assert sorted(api.SYMBOLS) == declared
     for name in declared:
         assert hasattr(lib, name), name
@@ -141,3 +141,40 @@ def test_rope_argument_errors(lib):
     assert lib.swa_rope_qk(p, 2, 4, MIS, FAKE, NULL, 0, NULL, NULL, NULL, 0, NULL) == 1
     assert lib.swa_rope_qk(p, 0, 4, FAKE, FAKE, NULL, 0, NULL, NULL, NULL, 0, NULL) == 0
     assert lib.swa_rope_qk(p, 2, 4, NULL, NULL, NULL, 0, NULL, NULL, NULL, 0, NULL) == 0
+
+
+def test_prefill_chunk_argument_errors(lib):
+    sl = _P(num_q_heads=8, num_kv_heads=2, window=512)
+    full = _P(num_q_heads=8, num_kv_heads=2, window=-1, rope_theta=5e6, rotary_dim=64)
+    # (B, S, pos0, q, k, v, gate, k_cache, v_cache, C, out, ws, ws_bytes, stream)
+    args = lambda C, pos0: (1, 256, pos0, FAKE, FAKE, FAKE, NULL, FAKE, FAKE, C, FAKE, FAKE, 1 << 34, NULL)
+    assert lib.swa_attn_prefill_chunk(sl, *args(256, 100)) == 1          # ring capacity != W
+    assert lib.swa_attn_prefill_chunk(full, *args(300, 100)) == 1        # capacity < pos0 + S
+    assert lib.swa_attn_prefill_chunk(full, 1, 256, -1, *args(4096, 0)[3:]) == 1   # negative pos0
+    assert lib.swa_attn_prefill_chunk(full, 1, 256, 0x7FFFFF00, *args(4096, 0)[3:]) == 1  # positions past 2^31
+    a = list(args(512, 100))
+    a[7] = NULL                                                          # k_cache missing
+    assert lib.swa_attn_prefill_chunk(sl, *a) == 1
+    a = list(args(512, 100))
+    a[8] = MIS                                                           # misaligned v_cache
+    assert lib.swa_attn_prefill_chunk(sl, *a) == 1
+    a = list(args(512, 100))
+    a[11], a[12] = NULL, 0                                               # workspace missing
+    assert lib.swa_attn_prefill_chunk(sl, *a) == 3
+    # nothing to do: returns before touching anything
+    assert lib.swa_attn_prefill_chunk(sl, 1, 0, 100, *([NULL] * 6), 512, NULL, NULL, 0, NULL) == 0
+
+
+def test_prefill_chunk_workspace_sizes(lib):
+    # sliding W 512, r 128: history min(pos0, 511) rows + the chunk, keys and
+    # values [B, h + S, Hkv, D] bf16 each, plus the table of S positions
+    sl = api.LayerParams(8, 2, 128, 512, 1e4, 128)
+    row = 2 * 128 * 2
+    up = lambda n: (n + 255) // 256 * 256
+    table = lambda S, half: ((S + 31) // 32) * ((half + 1) // 2) * 512
+    assert api.prefill_chunk_workspace_size(sl, 2, 300, 1000) == 2 * up(2 * (511 + 300) * row) + up(table(300, 64))
+    assert api.prefill_chunk_workspace_size(sl, 2, 300, 10) == 2 * up(2 * (10 + 300) * row) + up(table(300, 64))
+    # full layer: rotated chunk keys + table; without RoPE nothing at all
+    full = api.LayerParams(8, 2, 128, -1, 5e6, 64)
+    assert api.prefill_chunk_workspace_size(full, 2, 300, 5000) == up(2 * 300 * row) + up(table(300, 32))
+    assert api.prefill_chunk_workspace_size(api.LayerParams(8, 2, 128, -1, 0.0, 128), 2, 300, 5000) == 0

@@ -1,0 +1,98 @@
+"""swa_attn_prefill_chunk on the GPU: a sequence prefilled in several chunks
+against the KV cache gives the rows of the whole-sequence attention the
+oracle computes, and leaves the cache exactly as appending every token with
+swa_rope_qk would (ring: the last W positions; linear: all of them)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from full_gqa_attention_swa_b200 import api, inputs
+from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_chunks(cuda_device, p, B, bounds, seed, C, gate=True, L_inputs=None):
+    """Prefill positions bounds[0]..bounds[-1] chunk by chunk into a fresh
+    cache; returns the inputs (CPU, L_inputs >= bounds[-1] tokens), the
+    stacked outputs and the caches."""
+    L = bounds[-1] if L_inputs is None else L_inputs
+    d = inputs.prefill_inputs(B, L, p.num_q_heads, p.num_kv_heads, 128, seed, with_gate=gate)
+    dev = {k: (None if t is None else t.to(cuda_device)) for k, t in d.items()}
+    kc = torch.zeros(B, p.num_kv_heads, C, 128, dtype=torch.bfloat16, device=cuda_device)
+    vc = torch.zeros_like(kc)
+    outs = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        sl = slice(a, b)
+        g = None if dev["gate"] is None else dev["gate"][:, sl].contiguous()
+        out = api.attn_prefill_chunk(p, a, dev["q"][:, sl].contiguous(), dev["k"][:, sl].contiguous(),
+                                     dev["v"][:, sl].contiguous(), g, kc, vc)
+        outs.append(out)
+    torch.cuda.synchronize()
+    return d, torch.cat(outs, dim=1), kc, vc
+
+
+def _check(cuda_device, p, B, bounds, seed, C, gate=True):
+    d, out, kc, vc = _run_chunks(cuda_device, p, B, bounds, seed, C, gate)
+    ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]),
+                         None if d["gate"] is None else d["gate"].numpy())
+    assert_close(out, ref, f"chunks {bounds} W{p.window}")
+    # the cache equals appending the whole sequence in one swa_rope_qk call
+    L = bounds[-1]
+    kref = torch.zeros_like(kc)
+    vref = torch.zeros_like(vc)
+    k_all = d["k"].to(cuda_device).contiguous()
+    api.rope_qk(p, k=k_all, pos0=0, v=d["v"].to(cuda_device).contiguous(), k_cache=kref, v_cache=vref)
+    torch.cuda.synchronize()
+    slots = sorted({(pos % p.window) if p.window > 0 else pos for pos in range(max(0, L - (p.window if p.window > 0 else L)), L)})
+    idx = torch.tensor(slots, device=cuda_device)
+    assert torch.equal(kc[:, :, idx].view(torch.int16), kref[:, :, idx].view(torch.int16)), "k cache differs"
+    assert torch.equal(vc[:, :, idx].view(torch.int16), vref[:, :, idx].view(torch.int16)), "v cache differs"
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("bounds", [[0, 300], [0, 100, 137, 400], [0, 1, 2, 130, 131, 390], [0, 250, 640]],
+                         ids=["one", "odd", "tiny-steps", "long-chunk"])
+@pytest.mark.parametrize("W", [64, 100, 128, 200])
+def test_sliding_chunks(cuda_device, bounds, W):
+    """Ring cache: histories shorter than W - 1, chunks longer than W (only
+    the last W positions stay in the ring), offsets off the 128 grid."""
+    p = api.LayerParams(8, 2, 128, W, 1e4, 128)
+    _check(cuda_device, p, 2, bounds, seed=900 + W, C=W)
+
+
+@pytest.mark.parametrize("bounds", [[0, 300], [0, 100, 137, 400], [0, 1, 2, 130, 131, 390], [0, 256, 640]],
+                         ids=["one", "odd", "tiny-steps", "aligned"])
+@pytest.mark.parametrize("theta,r", [(5e6, 64), (0.0, 128)])
+def test_full_chunks(cuda_device, bounds, theta, r):
+    """Linear cache read in place: partial and no RoPE, offsets off the grid."""
+    p = api.LayerParams(8, 2, 128, -1, theta, r)
+    _check(cuda_device, p, 2, bounds, seed=950 + r, C=700)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (12, 1), (6, 2)])
+def test_chunk_gqa_groups_no_gate(cuda_device, Hq, Hkv):
+    _check(cuda_device, api.LayerParams(Hq, Hkv, 128, 96, 5e5, 32), 1, [0, 77, 300], seed=980 + Hq, C=96,
+           gate=False)
+    _check(cuda_device, api.LayerParams(Hq, Hkv, 128, -1, 1e4, 128), 1, [0, 200, 333], seed=990 + Hq, C=400,
+           gate=False)
+
+
+def test_decode_after_chunked_prefill(cuda_device):
+    """The cache a chunked prefill leaves feeds decode: the next token's
+    output equals the whole-sequence prefill's next row."""
+    p = api.LayerParams(8, 2, 128, 100, 1e4, 128)
+    B, L = 2, 301
+    d, _, kc, vc = _run_chunks(cuda_device, p, B, [0, 120, 300], seed=1234, C=100, L_inputs=L)
+    ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy(),
+                         rows=np.array([(b, L - 1, h) for b in range(B) for h in range(8)], np.int64))
+    q = d["q"][:, L - 1:L].to(cuda_device).contiguous()
+    k = d["k"][:, L - 1:L].to(cuda_device).contiguous()
+    v = d["v"][:, L - 1:L].to(cuda_device).contiguous()
+    api.rope_qk(p, q=q, k=k, pos0=L - 1, v=v, k_cache=kc, v_cache=vc)
+    lens = torch.full((B,), L, dtype=torch.int32, device=cuda_device)
+    out = api.attn_decode(p, q[:, 0].contiguous(), d["gate"][:, L - 1].to(cuda_device).contiguous(), kc, vc, lens, L)
+    torch.cuda.synchronize()
+    assert_close(out.reshape(B * 8, 128), ref.reshape(B * 8, 128), "decode after chunks")
+    check_no_device_error()
