@@ -56,6 +56,7 @@ class _Layer(ctypes.Structure):
         ("rope_theta", ctypes.c_double),
         ("rotary_dim", ctypes.c_int32),
         ("softmax_scale", ctypes.c_double),
+        ("inv_freq", ctypes.c_void_p),
     ]
 
 
@@ -65,6 +66,9 @@ class Layer:
 
     window: W >= 1 for a sliding layer (W keys including self), -1 for full.
     rope_theta: 0 means no rotary encoding.  softmax_scale <= 0: 1/sqrt(D).
+    inv_freq: rotary_dim/2 angular frequencies replacing theta^(-2k/r)
+    (caller-scaled RoPE, e.g. the full layers' YaRN of the Step explainer's
+    section 2.3), or None.
     """
 
     num_q_heads: int
@@ -74,10 +78,19 @@ class Layer:
     rope_theta: float = 10000.0
     rotary_dim: int = 128
     softmax_scale: float = 0.0
+    inv_freq: tuple = None
+
+    def __post_init__(self):
+        freq = None
+        if self.inv_freq is not None:
+            freq = np.ascontiguousarray(self.inv_freq, dtype=np.float64)
+            assert freq.shape == (self.rotary_dim // 2,)
+        object.__setattr__(self, "_freq", freq)  # kept alive with the layer
 
     def _c(self) -> _Layer:
         return _Layer(self.num_q_heads, self.num_kv_heads, self.head_dim, self.window,
-                      float(self.rope_theta), self.rotary_dim, float(self.softmax_scale))
+                      float(self.rope_theta), self.rotary_dim, float(self.softmax_scale),
+                      None if self._freq is None else self._freq.ctypes.data)
 
 
 _lib = None
@@ -91,6 +104,11 @@ def _load():
         lib.oracle_rope.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                     ctypes.c_void_p, ctypes.c_double, ctypes.c_int32, ctypes.c_void_p]
         lib.oracle_rope.restype = ctypes.c_int
+        lib.oracle_rope_table.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
+        lib.oracle_rope_table.restype = ctypes.c_int
+        lib.oracle_rope_vec_table.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_double]
+        lib.oracle_rope_vec_table.restype = None
         lib.oracle_prefill.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
@@ -154,6 +172,28 @@ def rope(x_bf16, pos, theta: float, rotary_dim: int) -> np.ndarray:
     out = np.empty((T, H, D), np.float64)
     _check(_load().oracle_rope(_ptr(x), T, H, D, _ptr(p), float(theta), rotary_dim, _ptr(out)), "rope")
     return out
+
+
+def rope_table(x_bf16, pos, inv_freq, rotary_dim: int) -> np.ndarray:
+    """RoPE of x[T, H, D] (bf16 bits) at positions pos[t] with pair k turned
+    at frequency inv_freq[k]; fp64 out."""
+    x = _u16(x_bf16)
+    T, H, D = x.shape
+    p = np.ascontiguousarray(pos, dtype=np.int64)
+    f = np.ascontiguousarray(inv_freq, dtype=np.float64)
+    assert p.shape == (T,) and f.shape == (rotary_dim // 2,)
+    out = np.empty((T, H, D), np.float64)
+    _check(_load().oracle_rope_table(_ptr(x), T, H, D, _ptr(p), _ptr(f), rotary_dim, _ptr(out)), "rope_table")
+    return out
+
+
+def rope_f64_table(x, p: float, inv_freq, rotary_dim: int) -> np.ndarray:
+    """Table-frequency RoPE of one fp64 head vector x[D] at position p."""
+    y = np.array(x, dtype=np.float64, copy=True)
+    f = np.ascontiguousarray(inv_freq, dtype=np.float64)
+    assert y.ndim == 1 and f.shape == (rotary_dim // 2,)
+    _load().oracle_rope_vec_table(_ptr(y), rotary_dim, _ptr(f), float(p))
+    return y
 
 
 def rope_f64(x, p: float, theta: float, rotary_dim: int) -> np.ndarray:

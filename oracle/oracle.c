@@ -50,6 +50,7 @@ typedef struct {
     double rope_theta;     /* 0 => no rotary position encoding */
     int32_t rotary_dim;    /* even, 0..head_dim */
     double softmax_scale;  /* <= 0 => 1/sqrt(head_dim) */
+    const double* inv_freq;  /* rotary_dim/2 angular frequencies, or NULL for theta^(-2k/r) */
 } oracle_layer;
 
 enum { ORACLE_OK = 0, ORACLE_BAD_ARG = 1, ORACLE_NO_MEM = 2 };
@@ -70,6 +71,9 @@ static int layer_ok(const oracle_layer* L) {
     if (L->window == 0 || L->window < -1) return 0;
     if (L->rotary_dim < 0 || L->rotary_dim > L->head_dim || (L->rotary_dim & 1)) return 0;
     if (L->rope_theta < 0.0) return 0;
+    if (L->inv_freq)
+        for (int32_t k = 0; k < L->rotary_dim / 2; ++k)
+            if (!(L->inv_freq[k] >= 0.0) || isinf(L->inv_freq[k])) return 0;
     return 1;
 }
 
@@ -93,6 +97,50 @@ void oracle_rope_vec(double* x, int32_t D, int32_t r, double theta, double p) {
         x[k + half] = b * c + a * s;
     }
     (void)D;
+}
+
+/* The same rotation with the frequency of pair k taken from a table
+ * (inv_freq[k], k < r/2) instead of theta^(-2k/r).  The Step explainer's
+ * section 2.3 gives the full layers a YaRN rope scaling (rope_type llama3,
+ * factor 2.0) whose remaining parameters it does not state, so the caller
+ * supplies the scaled frequencies; with inv_freq[k] = theta^(-2k/r) this is
+ * oracle_rope_vec. */
+void oracle_rope_vec_table(double* x, int32_t r, const double* inv_freq, double p) {
+    if (r == 0) return;
+    int32_t half = r / 2;
+    for (int32_t k = 0; k < half; ++k) {
+        double phi = p * inv_freq[k];
+        double c = cos(phi), s = sin(phi);
+        double a = x[k], b = x[k + half];
+        x[k] = a * c - b * s;
+        x[k + half] = b * c + a * s;
+    }
+}
+
+/* A layer's rotation: its frequency table if it has one, else theta. */
+static void layer_rope(const oracle_layer* L, double* x, double p) {
+    if (L->inv_freq)
+        oracle_rope_vec_table(x, L->rotary_dim, L->inv_freq, p);
+    else
+        oracle_rope_vec(x, L->head_dim, L->rotary_dim, L->rope_theta, p);
+}
+
+/* RoPE with a frequency table over a bf16 tensor x[T, H, D] (token t at
+ * position pos[t]); output out[T, H, D] in fp64. */
+int oracle_rope_table(const uint16_t* x, int64_t T, int32_t H, int32_t D, const int64_t* pos,
+                      const double* inv_freq, int32_t r, double* out) {
+    if (!x || !pos || !out || !inv_freq || T < 0 || H <= 0 || D <= 0 || r < 0 || r > D || (r & 1))
+        return ORACLE_BAD_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t h = 0; h < H; ++h) {
+            double* y = out + (t * H + h) * (int64_t)D;
+            const uint16_t* xs = x + (t * H + h) * (int64_t)D;
+            for (int32_t d = 0; d < D; ++d) y[d] = bf16_bits_to_f64(xs[d]);
+            oracle_rope_vec_table(y, r, inv_freq, (double)pos[t]);
+        }
+    }
+    return ORACLE_OK;
 }
 
 /* RoPE over a bf16 tensor x[T, H, D] whose token t sits at position pos[t].
@@ -200,7 +248,7 @@ int oracle_prefill(const oracle_layer* L, int32_t B, int32_t S, const uint16_t* 
                     krot[j * D + d] = bf16_bits_to_f64(ks[d]);
                     vd[j * D + d] = bf16_bits_to_f64(vs[d]);
                 }
-                oracle_rope_vec(krot + j * D, D, L->rotary_dim, L->rope_theta, (double)j);
+                layer_rope(L, krot + j * D, (double)j);
             }
             int err = 0;
 #pragma omp parallel
@@ -219,7 +267,7 @@ int oracle_prefill(const oracle_layer* L, int32_t B, int32_t S, const uint16_t* 
                         if (rb != b || rh / G != kvh) continue;
                         const uint16_t* qs = q + ((rb * S + ri) * Hq + rh) * D;
                         for (int32_t d = 0; d < D; ++d) qv[d] = bf16_bits_to_f64(qs[d]);
-                        oracle_rope_vec(qv, D, L->rotary_dim, L->rope_theta, (double)ri);
+                        layer_rope(L, qv, (double)ri);
                         /* the visible keys of row ri form the interval [j0, ri] */
                         int64_t j0 = (L->window > 0 && ri - (int64_t)L->window + 1 > 0)
                                          ? ri - (int64_t)L->window + 1 : 0;
@@ -262,8 +310,8 @@ int oracle_prefill_materialised(const oracle_layer* L, int32_t B, int32_t S, con
                     Qr[(int64_t)i * D + d] = bf16_bits_to_f64(q[(((int64_t)b * S + i) * Hq + h) * D + d]);
                     Kr[(int64_t)i * D + d] = bf16_bits_to_f64(k[(((int64_t)b * S + i) * Hkv + kvh) * D + d]);
                 }
-                oracle_rope_vec(Qr + (int64_t)i * D, D, L->rotary_dim, L->rope_theta, (double)i);
-                oracle_rope_vec(Kr + (int64_t)i * D, D, L->rotary_dim, L->rope_theta, (double)i);
+                layer_rope(L, Qr + (int64_t)i * D, (double)i);
+                layer_rope(L, Kr + (int64_t)i * D, (double)i);
             }
             /* scores with the mask as -inf */
             for (int32_t i = 0; i < S; ++i)

@@ -35,13 +35,15 @@ def _f64(t):
     return t.to(torch.float64)
 
 
-def _rope_complex(x, pos, theta, r):
-    """RoPE as multiplication of z_k = x_k + i x_{k+r/2} by exp(i p w_k)."""
-    if theta == 0 or r == 0:
+def _rope_complex(x, pos, theta, r, freq=None):
+    """RoPE as multiplication of z_k = x_k + i x_{k+r/2} by exp(i p w_k),
+    w_k = theta^(-2k/r) or freq[k]."""
+    if (theta == 0 and freq is None) or r == 0:
         return x.clone()
     half = r // 2
     k = torch.arange(half, dtype=torch.float64)
-    w = torch.tensor(float(theta), dtype=torch.float64) ** (-2.0 * k / r)
+    w = (torch.tensor(float(theta), dtype=torch.float64) ** (-2.0 * k / r) if freq is None
+         else torch.tensor(np.asarray(freq, np.float64)))
     ang = pos.to(torch.float64)[:, None] * w[None, :]                      # [S, half]
     rot = torch.polar(torch.ones_like(ang), ang)                             # e^{i ang}
     z = torch.complex(x[..., :half], x[..., half:r])                        # [..., S, H, half]
@@ -52,14 +54,14 @@ def _rope_complex(x, pos, theta, r):
     return y
 
 
-def _sdpa_reference(q, k, v, gate, window, theta, r):
+def _sdpa_reference(q, k, v, gate, window, theta, r, freq=None):
     """Library attention on the same inputs: torch SDPA in fp64 with an
     explicit boolean band mask from tril/triu; KV heads repeated per group."""
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     pos = torch.arange(S)
-    qr = _rope_complex(_f64(q), pos, theta, r)
-    kr = _rope_complex(_f64(k), pos, theta, r)
+    qr = _rope_complex(_f64(q), pos, theta, r, freq)
+    kr = _rope_complex(_f64(k), pos, theta, r, freq)
     G = Hq // Hkv
     kr = kr.repeat_interleave(G, dim=2)
     vv = _f64(v).repeat_interleave(G, dim=2)
@@ -368,3 +370,66 @@ def test_decode_new_token_override():
     vc[:, :, 20 % W] = vn
     ref = oracle.decode_f64(lay, q, d["gate"].numpy(), kc, vc, lens)
     np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-15)
+
+
+# ---- caller-supplied frequency tables (the full layers' YaRN scaling of the
+# Step explainer's section 2.3, whose parameters the page leaves open)
+
+def _scaled_table(theta, r, factor=2.0, keep_above=0.05, scale_below=0.002):
+    """A long-context table of the kind a caller passes: high frequencies
+    kept, low ones divided by `factor`, a linear blend in between."""
+    k = np.arange(r // 2, dtype=np.float64)
+    w = theta ** (-2.0 * k / r)
+    t = np.clip((np.log(w) - np.log(scale_below)) / (np.log(keep_above) - np.log(scale_below)), 0.0, 1.0)
+    return w / (factor * (1.0 - t) + t)
+
+
+def test_rope_table_of_theta_frequencies_is_theta_rope():
+    theta, r = 5e6, 64
+    table = theta ** (-2.0 * np.arange(r // 2) / r)
+    d = inputs.prefill_inputs(1, 40, 4, 2, 128, seed=71)
+    x = _bits(d["k"])[0]
+    pos = np.arange(40, dtype=np.int64)
+    np.testing.assert_allclose(oracle.rope_table(x, pos, table, r), oracle.rope(x, pos, theta, r),
+                               rtol=1e-12, atol=1e-12)
+    a = oracle.prefill(oracle.Layer(4, 2, 128, -1, theta, r), _bits(d["q"]), _bits(d["k"]), _bits(d["v"]),
+                       d["gate"].numpy())
+    b = oracle.prefill(oracle.Layer(4, 2, 128, -1, theta, r, inv_freq=tuple(table)), _bits(d["q"]),
+                       _bits(d["k"]), _bits(d["v"]), d["gate"].numpy())
+    np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-12)
+
+
+def test_rope_table_half_frequency_is_half_position():
+    """Halving every frequency turns a vector at position p exactly as the
+    unhalved table turns it at p / 2 (p even: both angles are one rounding
+    of p * w / 2)."""
+    rng = np.random.default_rng(3)
+    table = rng.uniform(1e-6, 1.0, 32)
+    for p in (2, 100, 4096, 131070):
+        x = rng.standard_normal(128)
+        np.testing.assert_array_equal(oracle.rope_f64_table(x, p, table / 2, 64),
+                                      oracle.rope_f64_table(x, p // 2, table, 64))
+
+
+@pytest.mark.parametrize("k", [0, 7, 31])
+def test_rope_table_unit_vector_angle(k):
+    """e_k turns by p * table[k] into the plane (e_k, e_(k + r/2))."""
+    table = _scaled_table(5e6, 64)
+    for p in (1, 17, 8191, 100003):
+        e = np.zeros(128)
+        e[k] = 1.0
+        y = oracle.rope_f64_table(e, p, table, 64)
+        expect = np.zeros(128)
+        expect[k] = math.cos(p * table[k])
+        expect[k + 32] = math.sin(p * table[k])
+        np.testing.assert_allclose(y, expect, atol=1e-12)
+
+
+@pytest.mark.parametrize("W", [-1, 24])
+def test_prefill_with_table_matches_torch_sdpa(W):
+    table = _scaled_table(5e6, 64)
+    d = inputs.prefill_inputs(2, 48, 6, 2, 128, seed=73)
+    lay = oracle.Layer(6, 2, 128, W, 5e6, 64, inv_freq=tuple(table))
+    got = oracle.prefill(lay, _bits(d["q"]), _bits(d["k"]), _bits(d["v"]), d["gate"].numpy())
+    ref = _sdpa_reference(d["q"], d["k"], d["v"], d["gate"], W, 5e6, 64, freq=table)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
