@@ -48,13 +48,16 @@ class _Params(ctypes.Structure):
         ("rope_theta", ctypes.c_double),
         ("rotary_dim", ctypes.c_int32),
         ("softmax_scale", ctypes.c_float),
+        ("inv_freq", ctypes.POINTER(ctypes.c_double)),
     ]
 
 
 @dataclass(frozen=True)
 class LayerParams:
     """swa_layer_params: window -1 = full causal; rope_theta 0 = no RoPE;
-    softmax_scale <= 0 = 1/sqrt(head_dim)."""
+    softmax_scale <= 0 = 1/sqrt(head_dim); inv_freq = rotary_dim/2 angular
+    frequencies replacing rope_theta^(-2k/rotary_dim) (a caller-scaled RoPE),
+    or None."""
 
     num_q_heads: int
     num_kv_heads: int
@@ -63,10 +66,19 @@ class LayerParams:
     rope_theta: float = 10000.0
     rotary_dim: int = 128
     softmax_scale: float = 0.0
+    inv_freq: tuple = None
 
     def c(self) -> _Params:
-        return _Params(self.num_q_heads, self.num_kv_heads, self.head_dim, self.window, float(self.rope_theta),
-                       self.rotary_dim, float(self.softmax_scale))
+        freq = None
+        if self.inv_freq is not None:
+            if len(self.inv_freq) != self.rotary_dim // 2:
+                raise ValueError(f"inv_freq holds {len(self.inv_freq)} values, rotary_dim/2 = {self.rotary_dim // 2}")
+            freq = (ctypes.c_double * len(self.inv_freq))(*map(float, self.inv_freq))
+        prm = _Params(self.num_q_heads, self.num_kv_heads, self.head_dim, self.window, float(self.rope_theta),
+                      self.rotary_dim, float(self.softmax_scale),
+                      None if freq is None else ctypes.cast(freq, ctypes.POINTER(ctypes.c_double)))
+        prm._freq = freq  # the table lives as long as the struct that points to it
+        return prm
 
 
 _lib = None

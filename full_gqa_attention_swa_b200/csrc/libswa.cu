@@ -55,10 +55,18 @@ swa_status check_layer(const swa_layer_params* p) {
   if (p->rotary_dim < 0 || p->rotary_dim > p->head_dim || (p->rotary_dim & 1))
     return fail(SWA_ERR_INVALID_ARG, "rotary_dim=%d (even, 0..head_dim)", p->rotary_dim);
   if (!isfinite(p->softmax_scale)) return fail(SWA_ERR_INVALID_ARG, "softmax_scale is not finite");
+  if (p->inv_freq)
+    for (int k = 0; k < p->rotary_dim / 2; ++k)
+      if (!(p->inv_freq[k] >= 0.0) || !isfinite(p->inv_freq[k]))
+        return fail(SWA_ERR_INVALID_ARG, "inv_freq[%d] must be finite and >= 0", k);
   return SWA_OK;
 }
 
-bool rotates(const swa_layer_params* p) { return p->rope_theta > 0.0 && p->rotary_dim > 0; }
+// A layer rotates when it has rotary dims and either a frequency table or a
+// positive base (theta 0 without a table: no rotary encoding).
+bool rotates(const swa_layer_params* p) {
+  return p->rotary_dim > 0 && (p->inv_freq != nullptr || p->rope_theta > 0.0);
+}
 
 float scale_log2(const swa_layer_params* p) {
   const double s = p->softmax_scale > 0.f ? (double)p->softmax_scale : 1.0 / sqrt((double)p->head_dim);
@@ -69,7 +77,7 @@ void fill_inv_freq(const swa_layer_params* p, double* inv_freq) {
   for (int k = 0; k < swa::kMaxRotaryHalf; ++k) inv_freq[k] = 0.0;
   if (!rotates(p)) return;
   for (int k = 0; k < p->rotary_dim / 2; ++k)
-    inv_freq[k] = pow(p->rope_theta, -2.0 * (double)k / (double)p->rotary_dim);
+    inv_freq[k] = p->inv_freq ? p->inv_freq[k] : pow(p->rope_theta, -2.0 * (double)k / (double)p->rotary_dim);
 }
 
 // ------------------------------------------------------------ TMA encoding

@@ -1,5 +1,6 @@
 // Rotary position encoding of Q and K (rotate-half pairs over the first
-// rotary_dim dims, angle p * theta^(-2k/rotary_dim)), with an optional append
+// rotary_dim dims, angle p * inv_freq[k]: theta^(-2k/rotary_dim), or the
+// caller's scaled frequencies), with an optional append
 // of the rotated key and the raw value into a KV cache (ring slot p mod W on
 // sliding layers, slot p on full layers).
 //
@@ -103,7 +104,7 @@ __device__ __forceinline__ void rotate_chunk(const uint16_t* row_src, uint16_t* 
   if (in_place) __syncwarp();
 }
 
-// cos and sin of a rotary angle.  The angle p * theta^(-2k/r) is formed in
+// cos and sin of a rotary angle.  The angle p * inv_freq[k] is formed in
 // fp64 and reduced to [-pi, pi] by subtracting the nearest multiple of 2*pi
 // (Cody-Waite reduction with 2*pi split into a double and its rounding
 // remainder), so its error stays near 1e-15 rad for any position below 2^31;

@@ -74,6 +74,14 @@ typedef struct swa_layer_params {
   double rope_theta;     /* >= 0; 0 means no rotary encoding */
   int32_t rotary_dim;    /* even, 0..head_dim; 0 means no rotary encoding */
   float softmax_scale;   /* > 0, or <= 0 for 1/sqrt(head_dim) */
+  /* Host pointer to rotary_dim/2 angular frequencies (each finite, >= 0)
+   * that replace rope_theta^(-2k/rotary_dim), or NULL.  For a scaled RoPE
+   * computed by the caller: the Step explainer's section 2.3 gives the full
+   * layers a YaRN scaling (llama3 style, factor 2.0) without its other
+   * parameters.  Read during the call only (copied into the launch); with a
+   * table the layer rotates whenever rotary_dim > 0, whatever rope_theta is.
+   * A zero-initialised struct leaves it NULL. */
+  const double* inv_freq;
 } swa_layer_params;
 
 /*
@@ -96,10 +104,10 @@ typedef struct swa_layer_params {
  *            call write the same slot; with explicit positions, no two tokens
  *            of one sequence in a call may map to the same slot (caller's
  *            promise).
- *   The angle is p * theta^(-2k/rotary_dim), evaluated in fp64; the
- *   rotation itself runs in fp32 and the result is rounded to bf16.
- *   With theta == 0 or rotary_dim == 0, q/k are left unchanged and the
- *   caches (if any) still receive k and v.
+ *   The angle is p * theta^(-2k/rotary_dim) (p * inv_freq[k] with a table),
+ *   evaluated in fp64; the rotation itself runs in fp32 and the result is
+ *   rounded to bf16.  With rotary_dim == 0, or theta == 0 and no table, q/k
+ *   are left unchanged and the caches (if any) still receive k and v.
  */
 SWA_API swa_status swa_rope_qk(const swa_layer_params* params, int32_t B, int32_t S, uint16_t* q, uint16_t* k,
                        const int32_t* pos, int32_t pos0, const uint16_t* v, uint16_t* k_cache,

@@ -12,7 +12,19 @@ RTOL = 1e-2
 
 def oracle_layer(p: api.LayerParams) -> oracle.Layer:
     return oracle.Layer(p.num_q_heads, p.num_kv_heads, p.head_dim, p.window, p.rope_theta, p.rotary_dim,
-                        p.softmax_scale)
+                        p.softmax_scale, p.inv_freq)
+
+
+def scaled_inv_freq(theta, r, factor=2.0, low=1.0, high=4.0, context=8192):
+    """A long-context frequency table a caller would pass as inv_freq: the
+    llama3-style rule (wavelengths shorter than context/high kept, longer
+    than context/low divided by factor, a linear blend between).  The pages
+    name this scaling for the full layers without its parameters, so the
+    values here are test inputs, not a reading of them."""
+    w = float(theta) ** (-2.0 * np.arange(r // 2) / r)
+    wavelen = 2 * np.pi / w
+    blend = np.clip((context / wavelen - low) / (high - low), 0.0, 1.0)
+    return tuple(float(x) for x in (1.0 - blend) * w / factor + blend * w)
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:

@@ -178,3 +178,23 @@ def test_prefill_chunk_workspace_sizes(lib):
     full = api.LayerParams(8, 2, 128, -1, 5e6, 64)
     assert api.prefill_chunk_workspace_size(full, 2, 300, 5000) == up(2 * 300 * row) + up(table(300, 32))
     assert api.prefill_chunk_workspace_size(api.LayerParams(8, 2, 128, -1, 0.0, 128), 2, 300, 5000) == 0
+
+
+def test_frequency_table(lib):
+    """A caller table makes a theta-0 layer rotate (workspace for keys and
+    the cos/sin table appears); a non-finite or negative entry is rejected
+    before any launch; the binding checks the table's length."""
+    table = tuple(0.5 ** k for k in range(32))
+    with_table = api.LayerParams(8, 2, 128, -1, 0.0, 64, inv_freq=table)
+    plain = api.LayerParams(8, 2, 128, -1, 0.0, 64)
+    assert api.prefill_workspace_size(plain, 1, 100) == 0
+    assert api.prefill_workspace_size(with_table, 1, 100) == (100 * 2 * 128 * 2 + 255) // 256 * 256 + 4 * 16 * 512
+    # rotary_dim 0 never rotates, table or not
+    assert api.prefill_workspace_size(api.LayerParams(8, 2, 128, -1, 0.0, 0, inv_freq=()), 1, 100) == 0
+    for bad in (float("nan"), float("inf"), -1e-3):
+        prm = api.LayerParams(8, 2, 128, -1, 1e4, 64, inv_freq=table[:31] + (bad,)).c()
+        st = lib.swa_attn_prefill(ctypes.byref(prm), 1, 128, FAKE, FAKE, FAKE, NULL, FAKE, FAKE, 1 << 30, NULL)
+        assert st == 1
+        assert "inv_freq[31]" in lib.swa_last_error_detail().decode()
+    with pytest.raises(ValueError):
+        api.LayerParams(8, 2, 128, -1, 1e4, 64, inv_freq=table[:30]).c()

@@ -8,7 +8,8 @@ import torch
 
 import oracle
 from full_gqa_attention_swa_b200 import api, configs, inputs
-from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer, prefill_rows_sample
+from gpu_helpers import (assert_close, bits, check_no_device_error, oracle_layer, prefill_rows_sample,
+                         scaled_inv_freq)
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +56,16 @@ def test_ragged_lengths(cuda_device, S, W):
 def test_rope_variants(cuda_device, theta, r):
     p = api.LayerParams(8, 2, 128, 200, theta, r)
     _check_all_rows(cuda_device, p, 1, 384, seed=300 + r)
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("W,theta,r", [(-1, 5e6, 64), (200, 1e4, 128), (-1, 0.0, 32)])
+def test_frequency_table(cuda_device, W, theta, r):
+    """Caller-scaled RoPE (the full layers' long-context scaling) through the
+    in-kernel Q rotation and the cos/sin table."""
+    table = scaled_inv_freq(theta if theta > 0 else 1e4, r)
+    p = api.LayerParams(8, 2, 128, W, theta, r, inv_freq=table)
+    _check_all_rows(cuda_device, p, 1, 384, seed=350 + r)
     check_no_device_error()
 
 

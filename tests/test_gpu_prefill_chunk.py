@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from full_gqa_attention_swa_b200 import api, inputs
-from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer
+from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer, scaled_inv_freq
 
 pytestmark = pytest.mark.gpu
 
@@ -79,12 +79,21 @@ def test_chunk_gqa_groups_no_gate(cuda_device, Hq, Hkv):
            gate=False)
 
 
-def test_decode_after_chunked_prefill(cuda_device):
+@pytest.mark.parametrize("W", [96, -1])
+def test_chunks_frequency_table(cuda_device, W):
+    table = scaled_inv_freq(5e6, 64)
+    p = api.LayerParams(8, 2, 128, W, 5e6, 64, inv_freq=table)
+    _check(cuda_device, p, 2, [0, 70, 333], seed=1010 + max(W, 0), C=96 if W > 0 else 400)
+
+
+@pytest.mark.parametrize("p,C", [(api.LayerParams(8, 2, 128, 100, 1e4, 128), 100),
+                                 (api.LayerParams(8, 2, 128, -1, 5e6, 64, inv_freq=scaled_inv_freq(5e6, 64)), 320)],
+                         ids=["sliding", "full-table"])
+def test_decode_after_chunked_prefill(cuda_device, p, C):
     """The cache a chunked prefill leaves feeds decode: the next token's
     output equals the whole-sequence prefill's next row."""
-    p = api.LayerParams(8, 2, 128, 100, 1e4, 128)
     B, L = 2, 301
-    d, _, kc, vc = _run_chunks(cuda_device, p, B, [0, 120, 300], seed=1234, C=100, L_inputs=L)
+    d, _, kc, vc = _run_chunks(cuda_device, p, B, [0, 120, 300], seed=1234, C=C, L_inputs=L)
     ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy(),
                          rows=np.array([(b, L - 1, h) for b in range(B) for h in range(8)], np.int64))
     q = d["q"][:, L - 1:L].to(cuda_device).contiguous()

@@ -6,7 +6,7 @@ import torch
 
 import oracle
 from full_gqa_attention_swa_b200 import api, inputs
-from gpu_helpers import assert_close, bits, check_no_device_error
+from gpu_helpers import assert_close, bits, check_no_device_error, scaled_inv_freq
 
 pytestmark = pytest.mark.gpu
 
@@ -26,6 +26,27 @@ def test_rope_in_place_matches_oracle(cuda_device, theta, r):
         if theta == 0 or r == 0:
             assert torch.equal(got.cpu(), src), name    # untouched, bit for bit
         assert_close(got.reshape(B * S, H, 128), ref, f"rope {name}")
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("theta,r", [(5e6, 64), (1e4, 128), (0.0, 32)])
+def test_rope_frequency_table_matches_oracle(cuda_device, theta, r):
+    """A caller table replaces theta^(-2k/r); with theta 0 the table still
+    rotates.  Positions up to 2^20 exercise the fp64 angle reduction."""
+    B, S, Hq, Hkv = 2, 29, 8, 2
+    table = scaled_inv_freq(theta if theta > 0 else 1e4, r)
+    p = api.LayerParams(Hq, Hkv, 128, -1, theta, r, inv_freq=table)
+    d = inputs.prefill_inputs(B, S, Hq, Hkv, 128, seed=47)
+    q = d["q"].to(cuda_device)
+    k = d["k"].to(cuda_device)
+    pos = torch.randint(0, 1 << 20, (B, S), generator=torch.Generator().manual_seed(5), dtype=torch.int32)
+    api.rope_qk(p, q=q, k=k, pos=pos.to(cuda_device))
+    torch.cuda.synchronize()
+    P = pos.numpy().reshape(-1).astype(np.int64)
+    for name, src, got, H in (("q", d["q"], q, Hq), ("k", d["k"], k, Hkv)):
+        ref = oracle.rope_table(bits(src).reshape(B * S, H, 128), P, np.array(table), r)
+        assert_close(got.reshape(B * S, H, 128), ref, f"rope table {name}")
+        assert not torch.equal(got.cpu(), src), name
     check_no_device_error()
 
 
