@@ -126,6 +126,11 @@ def _load():
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                           ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_decode_f64.restype = ctypes.c_int
+        lib.oracle_decode_mq.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+        lib.oracle_decode_mq.restype = ctypes.c_int
         lib.oracle_kv_cache_bytes.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                               ctypes.c_int32, ctypes.c_int32]
         lib.oracle_kv_cache_bytes.restype = ctypes.c_int64
@@ -290,6 +295,38 @@ def decode_f64(layer: Layer, q_rot, gate, k_cache, v_cache, seq_lens) -> np.ndar
     lay = layer._c()
     _check(_load().oracle_decode_f64(ctypes.byref(lay), B, _ptr(q), _ptr(g), _ptr(kc), _ptr(vc), C,
                                      _ptr(L), _ptr(out)), "decode_f64")
+    return out
+
+
+def decode_mq(layer: Layer, q_rot, gate, k_cache, v_cache, seq_lens, k_new, v_new, rows=None,
+              threads: int = 0) -> np.ndarray:
+    """Multi-query decode: T new tokens per sequence at positions
+    L_b - T .. L_b - 1 (L_b = seq_lens[b]); the bf16 cache [B,Hkv,C,D] holds
+    the L_b - T earlier tokens (ring slot p mod W, or slot p), the new
+    tokens' rotated keys / raw values are k_new / v_new [B,T,Hkv,D] bf16.
+
+    q_rot [B,T,Hq,D] fp64 (after RoPE); gate [B,T,Hq] float32 or None.
+    rows: int64 [n, 3] of (b, t, h) or None.  Returns fp64 [B,T,Hq,D] or [n, D].
+    """
+    kc, vc = _u16(k_cache), _u16(v_cache)
+    kn, vn = _u16(k_new), _u16(v_new)
+    B, Hkv, C, D = kc.shape
+    T = kn.shape[1]
+    assert kn.shape == (B, T, Hkv, D) and vn.shape == kn.shape
+    q = np.ascontiguousarray(q_rot, dtype=np.float64)
+    assert q.shape == (B, T, layer.num_q_heads, D)
+    g = None if gate is None else np.ascontiguousarray(gate, dtype=np.float32)
+    L = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    if rows is None:
+        r, n = None, 0
+        out = np.empty((B, T, layer.num_q_heads, D), np.float64)
+    else:
+        r = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+        n = r.shape[0]
+        out = np.empty((n, D), np.float64)
+    lay = layer._c()
+    _check(_load().oracle_decode_mq(ctypes.byref(lay), B, T, _ptr(q), _ptr(g), _ptr(kc), _ptr(vc), C, _ptr(L),
+                                    _ptr(kn), _ptr(vn), n, _ptr(r), _ptr(out), threads), "decode_mq")
     return out
 
 

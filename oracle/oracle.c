@@ -469,6 +469,99 @@ int oracle_decode_f64(const oracle_layer* L, int32_t B, const double* q_rot, con
     return ORACLE_OK;
 }
 
+/* Multi-query decode: T consecutive new tokens per sequence -- the extra
+ * next-token-prediction (MTP) layers of the Step spec card's config dump
+ * propose tokens that one attention call then checks -- at positions
+ * L0 .. L0 + T - 1, where L0 = seq_lens[b] - T.  The cache holds only the
+ * L0 earlier tokens (rotated keys, raw values): on a sliding layer a ring of
+ * W slots with position p in slot p mod W, so the last min(L0, W) positions
+ * are there (Step explainer section 2.2); on a full layer slots 0 .. L0 - 1.
+ * The new tokens' rotated keys and raw values come separately, k_new/v_new
+ * [B,T,Hkv,D] bf16 in position order.  Query t (position p = L0 + t) attends
+ * to the keys at positions j with p - W < j <= p (W = -1: 0 <= j <= p) --
+ * the band of every other query -- taking position j from the cache when
+ * j < L0, else new token j - L0.
+ * q_rot [B,T,Hq,D] fp64 (after RoPE); gate [B,T,Hq] or NULL;
+ * rows: n_rows (b, t, h) triples or NULL for all; out [n_rows or B*T*Hq, D]. */
+int oracle_decode_mq(const oracle_layer* L, int32_t B, int32_t T, const double* q_rot, const float* gate,
+                     const uint16_t* k_cache, const uint16_t* v_cache, int32_t C, const int32_t* seq_lens,
+                     const uint16_t* k_new, const uint16_t* v_new, int64_t n_rows, const int64_t* rows,
+                     double* out, int32_t n_threads) {
+    if (!layer_ok(L) || B < 0 || T < 1 || !q_rot || !k_cache || !v_cache || !seq_lens || !k_new || !v_new ||
+        !out || C <= 0 || (rows && n_rows < 0))
+        return ORACLE_BAD_ARG;
+    const int32_t Hq = L->num_q_heads, Hkv = L->num_kv_heads, D = L->head_dim;
+    const int32_t G = Hq / Hkv, W = L->window;
+    const double scale = layer_scale(L);
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t L0 = (int64_t)seq_lens[b] - T;
+        if (L0 < 0) return ORACLE_BAD_ARG;
+        if (W < 0 && L0 > C) return ORACLE_BAD_ARG;
+        if (W > 0 && C != W) return ORACLE_BAD_ARG;
+    }
+    const int64_t total = rows ? n_rows : (int64_t)B * T * Hq;
+    for (int64_t r = 0; rows && r < total; ++r)
+        if (rows[3 * r] < 0 || rows[3 * r] >= B || rows[3 * r + 1] < 0 || rows[3 * r + 1] >= T ||
+            rows[3 * r + 2] < 0 || rows[3 * r + 2] >= Hq)
+            return ORACLE_BAD_ARG;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+    int err = 0;
+#pragma omp parallel
+    {
+        double* kd = NULL;
+        double* vd = NULL;
+        double* sc = NULL;
+        int64_t cap = 0;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < total; ++r) {
+            const int64_t b = rows ? rows[3 * r] : r / ((int64_t)T * Hq);
+            const int64_t t = rows ? rows[3 * r + 1] : (r / Hq) % T;
+            const int64_t h = rows ? rows[3 * r + 2] : r % Hq;
+            const int64_t kvh = h / G;
+            const int64_t L0 = (int64_t)seq_lens[b] - T, p = L0 + t;
+            int64_t lo = 0;
+            for (; lo <= p && !visible(p, lo, W); ++lo) {
+            }
+            const int64_t n = p - lo + 1;
+            if (n > cap) {
+                free(kd); free(vd); free(sc);
+                kd = (double*)malloc(sizeof(double) * (size_t)n * D);
+                vd = (double*)malloc(sizeof(double) * (size_t)n * D);
+                sc = (double*)malloc(sizeof(double) * (size_t)n);
+                cap = (kd && vd && sc) ? n : 0;
+            }
+            if (!cap) {
+#pragma omp atomic write
+                err = 1;
+                continue;
+            }
+            for (int64_t j = lo; j <= p; ++j) {
+                const uint16_t *ks, *vs;
+                if (j < L0) {
+                    const int64_t slot = W > 0 ? j % W : j;
+                    ks = k_cache + ((b * Hkv + kvh) * C + slot) * D;
+                    vs = v_cache + ((b * Hkv + kvh) * C + slot) * D;
+                } else {
+                    ks = k_new + ((b * T + (j - L0)) * Hkv + kvh) * D;
+                    vs = v_new + ((b * T + (j - L0)) * Hkv + kvh) * D;
+                }
+                for (int32_t d = 0; d < D; ++d) {
+                    kd[(j - lo) * D + d] = bf16_bits_to_f64(ks[d]);
+                    vd[(j - lo) * D + d] = bf16_bits_to_f64(vs[d]);
+                }
+            }
+            const float* g = gate ? gate + (b * T + t) * Hq + h : NULL;
+            attend_row(q_rot + ((b * T + t) * Hq + h) * D, kd, vd, n, D, scale, g, out + r * D, sc);
+        }
+        free(kd); free(vd); free(sc);
+    }
+    return err ? ORACLE_NO_MEM : ORACLE_OK;
+}
+
 /* KV-cache footprint in bytes: tokens x kv-heads x head_dim x (K and V) x
  * bytes per element, summed over layers (Muse explainer, GQA section). */
 int64_t oracle_kv_cache_bytes(int64_t tokens, int32_t kv_heads, int32_t head_dim,

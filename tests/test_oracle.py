@@ -433,3 +433,92 @@ def test_prefill_with_table_matches_torch_sdpa(W):
     got = oracle.prefill(lay, _bits(d["q"]), _bits(d["k"]), _bits(d["v"]), d["gate"].numpy())
     ref = _sdpa_reference(d["q"], d["k"], d["v"], d["gate"], W, 5e6, 64, freq=table)
     np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+# ---- multi-query decode (T new tokens per sequence: the MTP layers' drafts
+# checked in one call; Step spec card config dump, Step explainer section 2.2)
+
+def _mq_setup(L, T, W, C=None, seed=81, Hq=6, Hkv=2, D=32):
+    """Inputs of one sequence of L tokens without RoPE (theta 0, so cached
+    keys are the raw bf16 keys); the cache holds the first L - T tokens."""
+    d = inputs.prefill_inputs(1, L, Hq, Hkv, D, seed=seed)
+    L0 = L - T
+    C = (W if W > 0 else L0 + 3) if C is None else C
+    kb, vb = _bits(d["k"])[0], _bits(d["v"])[0]            # [L, Hkv, D] uint16
+    kc = np.zeros((1, Hkv, C, D), np.uint16)
+    vc = np.zeros((1, Hkv, C, D), np.uint16)
+    for p in range(max(0, L0 - W) if W > 0 else 0, L0):
+        slot = p % W if W > 0 else p
+        kc[0, :, slot] = kb[p]
+        vc[0, :, slot] = vb[p]
+    return d, kc, vc, kb[None, L0:], vb[None, L0:]
+
+
+@pytest.mark.parametrize("L,T,W", [(40, 4, 8), (40, 3, 40), (7, 4, 16), (33, 2, 1), (5, 5, 8), (12, 4, 3),
+                                   (50, 1, 16), (64, 4, -1), (4, 4, -1)])
+def test_decode_mq_equals_prefill_rows(L, T, W):
+    """Each of the T queries equals the whole-sequence prefill's row at its
+    position: the cache part, the new-token part and the per-query band."""
+    Hq, Hkv, D = 6, 2, 32
+    d, kc, vc, kn, vn = _mq_setup(L, T, W)
+    lay = oracle.Layer(Hq, Hkv, D, W, 0.0, 0)
+    pre = oracle.prefill(lay, _bits(d["q"]), _bits(d["k"]), _bits(d["v"]), d["gate"].numpy())
+    q = oracle.bf16_bits_to_f64(_bits(d["q"]))[:, L - T:]
+    got = oracle.decode_mq(lay, q, d["gate"][:, L - T:].numpy(), kc, vc, np.array([L]), kn, vn)
+    np.testing.assert_allclose(got[0], pre[0, L - T:], rtol=1e-12, atol=1e-13)
+    rows = np.array([[0, T - 1, 5], [0, 0, 0], [0, T // 2, 3]], np.int64)
+    sub = oracle.decode_mq(lay, q, d["gate"][:, L - T:].numpy(), kc, vc, np.array([L]), kn, vn, rows=rows)
+    for i, (b, t, h) in enumerate(rows):
+        assert np.array_equal(sub[i], got[b, t, h])
+
+
+@pytest.mark.parametrize("W", [8, 16])
+def test_decode_mq_ignores_slots_outside_every_band(W):
+    """The oldest ring entry (position L0 - W) is outside every query's band,
+    and unfilled slots of a short ring are never read: NaN there changes
+    nothing."""
+    for L, T in ((40, 3), (9, 4)):
+        d, kc, vc, kn, vn = _mq_setup(L, T, W)
+        lay = oracle.Layer(6, 2, 32, W, 0.0, 0)
+        q = oracle.bf16_bits_to_f64(_bits(d["q"]))[:, L - T:]
+        ref = oracle.decode_mq(lay, q, None, kc, vc, np.array([L]), kn, vn)
+        L0 = L - T
+        nan = np.uint16(0x7FC0)
+        kc2, vc2 = kc.copy(), vc.copy()
+        dead = [(L0 - W) % W] if L0 >= W else list(range(L0, W))
+        for slot in dead:
+            kc2[0, :, slot] = nan
+            vc2[0, :, slot] = nan
+        got = oracle.decode_mq(lay, q, None, kc2, vc2, np.array([L]), kn, vn)
+        assert np.array_equal(got, ref)
+
+
+def test_decode_mq_one_query_is_decode_after_append():
+    """T = 1: the same result as appending the token to the cache and running
+    the one-query decode (ring and linear caches, several lengths)."""
+    B, Hq, Hkv, D, W = 3, 8, 2, 32, 16
+    lens = np.array([1, 16, 45], np.int32)
+    for window, C in ((W, W), (-1, 50)):
+        dd = inputs.decode_inputs(B, Hq, Hkv, D, C, seed=83)
+        new = inputs.prefill_inputs(B, 1, Hq, Hkv, D, seed=84)
+        kc, vc = _bits(dd["k_cache"]).copy(), _bits(dd["v_cache"]).copy()
+        kn, vn = _bits(new["k"]), _bits(new["v"])
+        lay = oracle.Layer(Hq, Hkv, D, window, 1e4, 32)
+        q = oracle.bf16_bits_to_f64(_bits(new["q"]))                 # [B,1,Hq,D]
+        got = oracle.decode_mq(lay, q, new["gate"].numpy(), kc, vc, lens, kn, vn)
+        for b, Lb in enumerate(lens):
+            slot = (Lb - 1) % W if window > 0 else Lb - 1
+            kc[b, :, slot] = kn[b, 0]
+            vc[b, :, slot] = vn[b, 0]
+        ref = oracle.decode(lay, q[:, 0], new["gate"][:, 0].numpy(), kc, vc, lens)
+        np.testing.assert_allclose(got[:, 0], ref, rtol=1e-13, atol=1e-14)
+
+
+def test_decode_mq_rejects_bad_lengths():
+    d, kc, vc, kn, vn = _mq_setup(10, 4, 8)
+    lay = oracle.Layer(6, 2, 32, 8, 0.0, 0)
+    q = oracle.bf16_bits_to_f64(_bits(d["q"]))[:, 6:]
+    with pytest.raises(ValueError):
+        oracle.decode_mq(lay, q, None, kc, vc, np.array([3]), kn, vn)          # fewer tokens than T
+    with pytest.raises(ValueError):
+        oracle.decode_mq(lay, q, None, kc[:, :, :4], vc[:, :, :4], np.array([10]), kn, vn)   # ring != W
