@@ -80,6 +80,16 @@ def decode_bytes(c, lens) -> int:
     return keys * c.Hkv * 128 * 2 * 2 + c.B * c.Hq * (128 * 2 * 2 + 4)
 
 
+def decode_mq_bytes(c, lens) -> int:
+    """Multi-query decode: the cached keys (the L - T earlier tokens, at most
+    W on a ring) read once per kv-head as K and V, plus q, gate and out of the
+    T new tokens and their k / v."""
+    W = c.window
+    ctx = [int(L) - c.T for L in lens]
+    keys = sum(min(n, W) if W > 0 else n for n in ctx)
+    return keys * c.Hkv * 128 * 2 * 2 + c.B * c.T * (c.Hq * (128 * 2 * 2 + 4) + c.Hkv * 128 * 2 * 2)
+
+
 # DRAM traffic per launch of the prefill attention kernel from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum; profiles/prefill_kernel_step37_sliding.md).
 # It describes only the kernel source it was taken on, so it is reported only
@@ -87,10 +97,10 @@ def decode_bytes(c, lens) -> int:
 PREFILL_TRAFFIC = {
     "workload": "step37_sliding_B1_S8192_Hq96_Hkv8_W512",
     "bytes": 402.3e6,
-    # prefill.cuh, ptx.cuh and swa_internal.cuh as captured; any change makes the figure stale
-    "source_sha256": "db0f5b00d682a47e4c3d7f3df87c987ef001879ed9a45969ece8bbae5d3d9345",
+    # prefill.cuh and ptx.cuh (the kernel and its PTX helpers) as captured; any change makes the figure stale
+    "source_sha256": "9767bf0b33fa98554812f667b18acbdbda37877106df8376d0bfc2ceaa139514",
 }
-PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh", "swa_internal.cuh")
+PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh")
 
 
 def prefill_source_digest():
@@ -352,6 +362,45 @@ def bench_decode(c, steps: int, warmup: int, dev):
     return ms, nbytes
 
 
+def bench_decode_mq(c, steps: int, warmup: int, dev):
+    from full_gqa_attention_swa_b200 import api
+
+    p = _layer(c)
+    lens = inputs.uniform_int(c.B, c.len_lo, c.len_hi, c.seed)
+    n_sets = 1 if c.window < 0 else N_ROTATE
+    sets = []
+    for r in range(n_sets):
+        d = inputs.decode_inputs(c.B, c.Hq, c.Hkv, 128, c.capacity, c.seed + r, device=dev)
+        new = inputs.prefill_inputs(c.B, c.T, c.Hq, c.Hkv, 128, c.seed + 100 + r, device=dev)
+        sets.append((d, new))
+    lens_d = lens.to(dev)
+    max_len = int(lens.max())
+    out = torch.empty(c.B, c.T, c.Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(api.decode_mq_workspace_size(p, c.B, c.T, max_len), 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        d, new = sets[i % n_sets]
+        api.attn_decode_mq(p, new["q"], new["gate"], new["k"], new["v"], d["k_cache"], d["v_cache"], lens_d,
+                           max_len, out=out, workspace=ws, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / steps
+    nbytes = decode_mq_bytes(c, lens.tolist())
+    del sets
+    torch.cuda.empty_cache()
+    return ms, nbytes
+
+
 # --------------------------------------------------------------- CPU oracle
 
 def oracle_sample_rate(c, budget_s: float, threads: int = 0):
@@ -390,7 +439,7 @@ def main():
     ap.add_argument("--workload", default=configs.STEP_SLIDING.name, choices=sorted(configs.PREFILL))
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--only", choices=["all", "prefill", "decode_sliding", "decode_full", "chunk_sliding",
-                                       "chunk_full"], default="all",
+                                       "chunk_full", "decode_mq_sliding", "decode_mq_full"], default="all",
                     help="run one leg only (profiling); prints that leg's own JSON line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
@@ -462,10 +511,15 @@ def main():
         return
 
     if args.only.startswith("decode"):
-        dc = configs.DECODE_SLIDING if args.only == "decode_sliding" else configs.DECODE_FULL
+        mq = args.only.startswith("decode_mq")
+        if mq:
+            dc = configs.MQ_SLIDING if args.only == "decode_mq_sliding" else configs.MQ_FULL
+        else:
+            dc = configs.DECODE_SLIDING if args.only == "decode_sliding" else configs.DECODE_FULL
         if dist is not None:
             dist.barrier()
-        d_ms, nbytes = bench_decode(dc, max(args.steps, 1), max(args.warmup, 3), dev)
+        run = bench_decode_mq if mq else bench_decode
+        d_ms, nbytes = run(dc, max(args.steps, 1), max(args.warmup, 3), dev)
         d_ms = max_over_ranks(d_ms, dist, dev)
         gbs = nbytes * world / (d_ms / 1e3) / 1e9
         if rank == 0:
@@ -511,6 +565,13 @@ def main():
                 extra[dc.name] = {"ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                                   "peak_source": f"{peak_src} hbm copy"}
             line["decode"] = extra
+            mqs = {}
+            for mc in (configs.MQ_SLIDING, configs.MQ_FULL):
+                d_ms, nbytes = bench_decode_mq(mc, 200 if mc.window > 0 else 10, 3, dev)
+                gbs = nbytes / (d_ms / 1e3) / 1e9
+                mqs[mc.name] = {"ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                                "peak_source": f"{peak_src} hbm copy"}
+            line["decode_mq"] = mqs
             chunks = {}
             for cc in (configs.CHUNK_SLIDING, configs.CHUNK_FULL):
                 c_ms = bench_prefill_chunk(cc, 20 if cc.window > 0 else 5, 3, dev)

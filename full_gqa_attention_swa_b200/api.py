@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "SWA_OK", 1: "SWA_ERR_INVALID_ARG", 2: "SWA_ERR_UNSUPPORTED",
 SYMBOLS = ("swa_rope_qk", "swa_prefill_workspace_size", "swa_attn_prefill", "swa_decode_workspace_size",
            "swa_attn_decode", "swa_kv_cache_bytes", "swa_status_string", "swa_last_error_detail",
            "swa_device_error", "swa_version", "swa_attn_decode_no_alloc", "swa_prefill_chunk_workspace_size",
-           "swa_attn_prefill_chunk")
+           "swa_attn_prefill_chunk", "swa_decode_mq_workspace_size", "swa_attn_decode_mq")
 
 # bytes of the static device array behind swa_attn_decode_no_alloc
 NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -120,6 +120,10 @@ def load(path: str = LIB_PATH):
     lib.swa_prefill_chunk_workspace_size.restype = sz
     lib.swa_attn_prefill_chunk.argtypes = [P, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.swa_attn_prefill_chunk.restype = ctypes.c_int
+    lib.swa_decode_mq_workspace_size.argtypes = [P, i32, i32, i32]
+    lib.swa_decode_mq_workspace_size.restype = sz
+    lib.swa_attn_decode_mq.argtypes = [P, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, i32, vp, vp, sz, vp]
+    lib.swa_attn_decode_mq.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -270,6 +274,39 @@ def attn_decode(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens, max_len
     _check(load().swa_attn_decode(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache), _ptr(v_cache), C,
                                   _ptr(seq_lens), int(max_len), _ptr(out), _ptr(workspace), nbytes,
                                   _stream(stream)))
+    return out
+
+
+def decode_mq_workspace_size(layer: LayerParams, B: int, T: int, max_len: int) -> int:
+    return int(load().swa_decode_mq_workspace_size(ctypes.byref(layer.c()), B, T, max_len))
+
+
+def attn_decode_mq(layer: LayerParams, q, gate, k_new, v_new, k_cache, v_cache, seq_lens, max_len: int, out=None,
+                   workspace=None, stream=None):
+    """swa_attn_decode_mq: T new tokens per sequence in one call.  q [B,T,Hq,D]
+    and k_new [B,T,Hkv,D] already rotated, v_new [B,T,Hkv,D], gate [B,T,Hq]
+    fp32 or None; the caches [B,Hkv,C,D] hold the L - T earlier tokens only;
+    seq_lens [B] int32 (device) counts the new tokens.  Returns out [B,T,Hq,D]."""
+    B, T = q.shape[0], q.shape[1]
+    D = layer.head_dim
+    C = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (B, T, layer.num_q_heads, D))
+    _need(gate, "gate", torch.float32, (B, T, layer.num_q_heads))
+    _need(k_new, "k_new", torch.bfloat16, (B, T, layer.num_kv_heads, D))
+    _need(v_new, "v_new", torch.bfloat16, (B, T, layer.num_kv_heads, D))
+    _need(k_cache, "k_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, (B, T, layer.num_q_heads, D))
+    need = decode_mq_workspace_size(layer, B, T, max_len)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().swa_attn_decode_mq(ctypes.byref(layer.c()), B, T, _ptr(q), _ptr(gate), _ptr(k_new), _ptr(v_new),
+                                     _ptr(k_cache), _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
+                                     _ptr(workspace), nbytes, _stream(stream)))
     return out
 
 

@@ -64,6 +64,25 @@ class ChunkLayer:
     seed: int
 
 
+@dataclass(frozen=True)
+class MultiQueryLayer:
+    """Multi-query decode: T new tokens per sequence (lengths counting them
+    uniform in [len_lo, len_hi]); the cache holds the earlier tokens."""
+    name: str
+    B: int
+    T: int
+    Hq: int
+    Hkv: int
+    D: int
+    window: int
+    theta: float
+    rotary_dim: int
+    len_lo: int
+    len_hi: int
+    capacity: int
+    seed: int
+
+
 # tiny oracle case: B1 S256 Hq8 Hkv1 W64, theta 1e4 on all 128 dims
 TINY = PrefillLayer("tiny_B1_S256_Hq8_Hkv1_W64", 1, 256, 8, 1, 128, 64, 1e4, 128, 1000)
 
@@ -87,6 +106,14 @@ DECODE_SLIDING = DecodeLayer("decode_sliding_B64_Hq96_Hkv8_W512", 64, 96, 8, 128
 DECODE_FULL = DecodeLayer("decode_full_B64_Hq64_Hkv8", 64, 64, 8, 128, WINDOW_FULL, 5e6, 64,
                           4096, 131072, 131072, 1004)
 
+# multi-query decode of the Step layers: the token being decoded plus the
+# three tokens that the spec card's three MTP layers (architecture notes)
+# propose, T = 4
+MQ_SLIDING = MultiQueryLayer("decode_mq_sliding_B64_T4_Hq96_Hkv8_W512", 64, 4, 96, 8, 128, 512, 1e4, 128,
+                             4096, 131072, 512, 1007)
+MQ_FULL = MultiQueryLayer("decode_mq_full_B64_T4_Hq64_Hkv8", 64, 4, 64, 8, 128, WINDOW_FULL, 5e6, 64,
+                          4096, 131072, 131072, 1008)
+
 # continued prefill: the second half of the Step sliding and full prefills,
 # chunked against the cache the first half left
 CHUNK_SLIDING = ChunkLayer("step37_sliding_chunk_B1_pos4096_S4096_Hq96_Hkv8_W512", 1, 4096, 4096, 96, 8, 128,
@@ -97,3 +124,4 @@ CHUNK_FULL = ChunkLayer("step37_full_chunk_B1_pos16384_S16384_Hq64_Hkv8", 1, 163
 PREFILL = {c.name: c for c in (TINY, STEP_SLIDING, STEP_FULL, MUSE_SLIDING, MUSE_FULL)}
 CHUNK = {c.name: c for c in (CHUNK_SLIDING, CHUNK_FULL)}
 DECODE = {c.name: c for c in (DECODE_SLIDING, DECODE_FULL)}
+MULTI_QUERY = {c.name: c for c in (MQ_SLIDING, MQ_FULL)}

@@ -13,6 +13,7 @@
 #include "swa_internal.cuh"
 
 #include "decode.cuh"
+#include "decode_mq.cuh"
 #include "kv_gather.cuh"
 #include "prefill.cuh"
 #include "rope.cuh"
@@ -218,6 +219,36 @@ DecodePlan plan_decode(const swa_layer_params* p, int B, int max_len) {
   }
   if (pl.splits > 1) {
     const size_t rows = (size_t)B * p->num_q_heads * pl.splits;
+    pl.o_bytes = round_up(rows * kHeadDim * sizeof(float), 256);
+    pl.ml_bytes = round_up(rows * sizeof(float2), 256);
+  }
+  pl.total = pl.o_bytes + pl.ml_bytes;
+  return pl;
+}
+
+// Multi-query decode: the same split policy over the cached keys (the new
+// tokens ride on the last split), with the kernel's resident CTAs per SM.
+DecodePlan plan_decode_mq(const swa_layer_params* p, int B, int T, int max_len) {
+  DecodePlan pl{};
+  const long long kb = swa::kDecodeKeyBlock;
+  const long long ctx = max_len - T > 0 ? max_len - T : 0;
+  const long long n_vis = p->window > 0 ? (ctx < p->window ? ctx : p->window) : ctx;
+  const int rows = T * (p->num_q_heads / p->num_kv_heads);
+  const long long slots = 148LL * swa::decode_mq_ctas_per_sm(rows), items = (long long)B * p->num_kv_heads;
+  long long c = (items * n_vis + slots - 1) / slots;
+  c = (c + kb - 1) / kb * kb;
+  if (c < 256) c = 256;
+  if (c > 4096) c = 4096;
+  if (2 * items >= slots && n_vis <= 4096) c = n_vis;
+  if (c >= n_vis) {
+    pl.chunk = (int)(n_vis > 0 ? (n_vis + kb - 1) / kb * kb : kb);
+    pl.splits = 1;
+  } else {
+    pl.chunk = (int)c;
+    pl.splits = (int)((n_vis + c - 1) / c);
+  }
+  if (pl.splits > 1) {
+    const size_t rows = (size_t)B * T * p->num_q_heads * pl.splits;
     pl.o_bytes = round_up(rows * kHeadDim * sizeof(float), 256);
     pl.ml_bytes = round_up(rows * sizeof(float2), 256);
   }
@@ -561,6 +592,61 @@ swa_status swa_attn_decode(const swa_layer_params* p, int32_t B, const uint16_t*
   a.part_o = pl.splits > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
   a.part_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace) + pl.o_bytes) : nullptr;
   st = cuda_status(swa::launch_decode(a, km, vm, (cudaStream_t)stream), "decode launch");
+  return st == SWA_OK ? ok() : st;
+}
+
+size_t swa_decode_mq_workspace_size(const swa_layer_params* p, int32_t B, int32_t T, int32_t max_len) {
+  if (check_layer(p) != SWA_OK || B < 0 || T < 1 || T > swa::kDecodeMqMaxT || max_len < T) return 0;
+  return plan_decode_mq(p, B, T, max_len).total;
+}
+
+swa_status swa_attn_decode_mq(const swa_layer_params* p, int32_t B, int32_t T, const uint16_t* q, const float* gate,
+                              const uint16_t* k_new, const uint16_t* v_new, const uint16_t* k_cache,
+                              const uint16_t* v_cache, int32_t cache_capacity, const int32_t* seq_lens,
+                              int32_t max_len, uint16_t* out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  swa_status st = check_layer(p);
+  if (st != SWA_OK) return st;
+  if (B < 0) return fail(SWA_ERR_INVALID_ARG, "B=%d must be >= 0", B);
+  if (T < 1) return fail(SWA_ERR_INVALID_ARG, "T=%d must be >= 1", T);
+  if (B == 0) return ok();
+  const int Hq = p->num_q_heads, Hkv = p->num_kv_heads, G = Hq / Hkv;
+  if (T > swa::kDecodeMqMaxT || (long long)T * G > swa::kDecodeMqMaxRows)
+    return fail(SWA_ERR_UNSUPPORTED, "multi-query decode supports T <= %d and T * G <= %d (T=%d, G=%d)",
+                swa::kDecodeMqMaxT, swa::kDecodeMqMaxRows, T, G);
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !seq_lens || !out)
+    return fail(SWA_ERR_INVALID_ARG, "q, k_new, v_new, k_cache, v_cache, seq_lens and out must be non-NULL");
+  const void* ptrs[] = {q, gate, k_new, v_new, k_cache, v_cache, seq_lens, out, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(SWA_ERR_INVALID_ARG, "tensor pointer %p is not 16-byte aligned", ptr);
+  if (cache_capacity < 1) return fail(SWA_ERR_INVALID_ARG, "cache_capacity=%d", cache_capacity);
+  if (p->window > 0 && cache_capacity != p->window)
+    return fail(SWA_ERR_INVALID_ARG, "sliding layer: cache_capacity=%d must equal window=%d", cache_capacity,
+                p->window);
+  if (max_len < T) return fail(SWA_ERR_INVALID_ARG, "max_len=%d must be >= T=%d", max_len, T);
+  if (p->window < 0 && max_len - T > cache_capacity)
+    return fail(SWA_ERR_INVALID_ARG, "full layer: max_len - T = %d cached tokens exceed cache_capacity=%d",
+                max_len - T, cache_capacity);
+  if (B > 65535 || Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B=%d or Hkv=%d too large", B, Hkv);
+  const DecodePlan pl = plan_decode_mq(p, B, T, max_len);
+  if (pl.total > 0) {
+    if (!workspace) return fail(SWA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", pl.total);
+    if (workspace_bytes < pl.total)
+      return fail(SWA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, pl.total);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(SWA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  CUtensorMap km, vm;
+  if ((st = encode_cache(&km, k_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
+  if ((st = encode_cache(&vm, v_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
+  swa::DecodeMqArgs a{};
+  a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.window = p->window; a.capacity = cache_capacity;
+  a.scale_log2 = scale_log2(p);
+  a.q = q; a.gate = gate; a.k_new = k_new; a.v_new = v_new; a.seq_lens = seq_lens; a.out = out;
+  a.chunk = pl.chunk; a.max_splits = pl.splits;
+  a.part_o = pl.splits > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
+  a.part_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace) + pl.o_bytes) : nullptr;
+  st = cuda_status(swa::launch_decode_mq(a, km, vm, (cudaStream_t)stream), "multi-query decode launch");
   return st == SWA_OK ? ok() : st;
 }
 

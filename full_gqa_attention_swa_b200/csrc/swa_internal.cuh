@@ -18,6 +18,7 @@ enum : int {
   kErrPrefill = 100,
   kErrDecode = 200,
   kErrRope = 300,
+  kErrDecodeMq = 400,
 };
 
 // ------------------------------------------------------------------ RoPE
@@ -119,5 +120,33 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& k_map, const C
                           cudaStream_t stream);
 
 constexpr int kDecodeKeyBlock = 32;   // keys per pipeline stage
+
+// --------------------------------------------------- multi-query decode
+
+constexpr int kDecodeMqMaxT = 16;      // new tokens per sequence
+constexpr int kDecodeMqMaxRows = 64;   // T * G (query, head) rows per kv-head
+// resident multi-query decode CTAs per SM for T * G rows (sizes the split plan)
+constexpr int decode_mq_ctas_per_sm(int rows) { return rows <= 48 ? 3 : 2; }
+
+struct DecodeMqArgs {
+  int B, T, Hq, Hkv, G;
+  int window;                // W >= 1 (ring of W slots) or -1 (linear)
+  int capacity;              // C
+  float scale_log2;
+  const uint16_t* q;         // [B,T,Hq,D] rotated
+  const float* gate;         // [B,T,Hq] or nullptr
+  const uint16_t* k_new;     // [B,T,Hkv,D] rotated keys of the new tokens
+  const uint16_t* v_new;     // [B,T,Hkv,D]
+  const int32_t* seq_lens;   // [B], counting the T new tokens
+  uint16_t* out;             // [B,T,Hq,D]
+  int chunk;                 // cache keys per split (multiple of the key block)
+  int max_splits;
+  float* part_o;             // [B*T*Hq][max_splits][D] (split mode)
+  float2* part_ml;           // [B*T*Hq][max_splits]
+};
+
+// kv maps as for launch_decode; m_tiles = ceil(T*G / 16) selects the kernel.
+cudaError_t launch_decode_mq(const DecodeMqArgs& a, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                             cudaStream_t stream);
 
 }  // namespace swa

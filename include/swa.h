@@ -218,6 +218,53 @@ SWA_API swa_status swa_attn_decode(const swa_layer_params* params, int32_t B, co
                            size_t workspace_bytes, void* stream);
 
 /*
+ * swa_decode_mq_workspace_size -- bytes of workspace swa_attn_decode_mq needs
+ * for B sequences of T new tokens whose lengths (new tokens included) are at
+ * most max_len.  Returns 0 when no workspace is needed or parameters are
+ * invalid.
+ */
+SWA_API size_t swa_decode_mq_workspace_size(const swa_layer_params* params, int32_t B, int32_t T,
+                                            int32_t max_len);
+
+/*
+ * swa_attn_decode_mq -- T new tokens per sequence attend in one call, each
+ * through its own band: the check of tokens proposed by multi-token-
+ * prediction (MTP) layers ("Step-3.7-Flash" spec card, architecture notes:
+ * three such layers speed up decoding) or any other speculative draft.  Band and cache rule: Step explainer section 2.2; gate:
+ * section 2.3.
+ *
+ *   T        1 <= T <= 16 new tokens per sequence, and T * (Hq / Hkv) <= 64
+ *            (SWA_ERR_UNSUPPORTED otherwise).
+ *   q        [B, T, Hq, D] bf16, ALREADY rotated (positions L_b - T .. L_b - 1)
+ *   gate     [B, T, Hq] fp32 logits, or NULL
+ *   k_new    [B, T, Hkv, D] bf16, the new tokens' ALREADY rotated keys
+ *   v_new    [B, T, Hkv, D] bf16, their values
+ *   k_cache, v_cache  [B, Hkv, C, D] bf16 holding the L_b - T EARLIER tokens
+ *            only: a ring of C = W slots on a sliding layer (position p in
+ *            slot p mod W), slots 0 .. L_b - T - 1 on a full layer
+ *            (C >= max_len - T).  The new tokens are NOT in the cache, so a
+ *            rejected draft never overwrites a ring slot; append the accepted
+ *            ones afterwards with swa_rope_qk (rotary_dim = 0 in a copy of the
+ *            parameters appends already rotated keys unchanged).
+ *   seq_lens [B] int32 device, L_b >= T, counting the T new tokens.  Query t
+ *            sits at position L_b - T + t and sees the keys j with
+ *            p - W < j <= p: cached ones and new tokens 0 .. t.  A sequence
+ *            with L_b < T (or, full layer, L_b - T > C) records device error
+ *            403 (404) and its rows are left unwritten.
+ *   max_len  host-side upper bound of seq_lens (sizes the split grid).
+ *   out      [B, T, Hq, D] bf16
+ *   workspace / workspace_bytes: at least swa_decode_mq_workspace_size()
+ *            bytes (may be NULL when that is 0); overwritten.
+ *   Cache slots outside every query's band (unfilled slots, the oldest ring
+ *   entry) are never read as values: they may hold anything, including NaN.
+ */
+SWA_API swa_status swa_attn_decode_mq(const swa_layer_params* params, int32_t B, int32_t T, const uint16_t* q,
+                                      const float* gate, const uint16_t* k_new, const uint16_t* v_new,
+                                      const uint16_t* k_cache, const uint16_t* v_cache, int32_t cache_capacity,
+                                      const int32_t* seq_lens, int32_t max_len, uint16_t* out, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/*
  * swa_kv_cache_bytes -- bytes of one layer's K and V cache for `batch`
  * sequences of up to `context` tokens: batch x Hkv x C x D x 2 (K and V) x 2
  * (bf16), with C = min(context, W) on a sliding layer and C = context on a

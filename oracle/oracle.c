@@ -469,9 +469,10 @@ int oracle_decode_f64(const oracle_layer* L, int32_t B, const double* q_rot, con
     return ORACLE_OK;
 }
 
-/* Multi-query decode: T consecutive new tokens per sequence -- the extra
- * next-token-prediction (MTP) layers of the Step spec card's config dump
- * propose tokens that one attention call then checks -- at positions
+/* Multi-query decode: T consecutive new tokens per sequence -- the Step spec
+ * card's architecture notes list three extra multi-token-prediction (MTP)
+ * layers that speed up decoding; the tokens they propose are checked by one
+ * attention call -- at positions
  * L0 .. L0 + T - 1, where L0 = seq_lens[b] - T.  The cache holds only the
  * L0 earlier tokens (rotated keys, raw values): on a sliding layer a ring of
  * W slots with position p in slot p mod W, so the last min(L0, W) positions

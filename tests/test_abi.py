@@ -33,7 +33,7 @@ def _P(**kw):
 
 def test_exports_every_declared_symbol(lib):
     declared = _declared()
-    assert len(declared) == len(api.SYMBOLS) == 13
+    assert len(declared) == len(api.SYMBOLS) == 15
     assert sorted(api.SYMBOLS) == declared
     for name in declared:
         assert hasattr(lib, name), name
@@ -198,3 +198,42 @@ def test_frequency_table(lib):
         assert "inv_freq[31]" in lib.swa_last_error_detail().decode()
     with pytest.raises(ValueError):
         api.LayerParams(8, 2, 128, -1, 1e4, 64, inv_freq=table[:30]).c()
+
+
+def test_decode_mq_argument_errors(lib):
+    sl = _P(num_q_heads=96, num_kv_heads=8, window=512)
+    full = _P(num_q_heads=64, num_kv_heads=8, window=-1, rope_theta=5e6, rotary_dim=64)
+    # (B, T, q, gate, k_new, v_new, k_cache, v_cache, C, seq_lens, max_len, out, ws, ws_bytes, stream)
+    args = lambda T, C, max_len: (4, T, FAKE, NULL, FAKE, FAKE, FAKE, FAKE, C, FAKE, max_len, FAKE, FAKE,
+                                  1 << 34, NULL)
+    assert lib.swa_attn_decode_mq(sl, *args(4, 256, 600)) == 1             # ring capacity != W
+    assert lib.swa_attn_decode_mq(full, *args(4, 1000, 1005)) == 1         # max_len - T > capacity
+    assert lib.swa_attn_decode_mq(full, *args(4, 1000, 3)) == 1            # max_len < T
+    assert lib.swa_attn_decode_mq(full, *args(0, 1000, 10)) == 1           # T < 1
+    assert lib.swa_attn_decode_mq(full, *args(9, 1000, 100)) == 2          # T * G = 72 > 64
+    assert lib.swa_attn_decode_mq(sl, *args(17, 512, 100)) == 2            # T > 16
+    assert lib.swa_attn_decode_mq(_P(num_q_heads=34, num_kv_heads=1), *args(2, 64, 10)) == 2   # 68 rows
+    a = list(args(4, 1000, 1004))
+    a[4] = MIS                                                             # misaligned k_new
+    assert lib.swa_attn_decode_mq(full, *a) == 1
+    a = list(args(4, 1000, 1004))
+    a[5] = NULL                                                            # v_new missing
+    assert lib.swa_attn_decode_mq(full, *a) == 1
+    a = list(args(4, 131072, 131072))
+    a[12], a[13] = NULL, 0                                                 # workspace missing
+    assert lib.swa_attn_decode_mq(full, *a) == 3
+    assert lib.swa_attn_decode_mq(sl, 0, 4, *([NULL] * 6), 512, NULL, 600, NULL, NULL, 0, NULL) == 0
+
+
+def test_decode_mq_workspace_sizes(lib):
+    # sliding B64 (one split: 512 (sequence, kv-head) pairs fill the SM slots)
+    sl = api.LayerParams(96, 8, 128, 512, 1e4, 128)
+    assert api.decode_mq_workspace_size(sl, 64, 4, 131072) == 0
+    # full B64 T4: split-K partials for B * T * Hq rows
+    full = api.LayerParams(64, 8, 128, -1, 5e6, 64)
+    ws = api.decode_mq_workspace_size(full, 64, 4, 131072)
+    rows = 64 * 4 * 64
+    splits = ws // (rows * (128 * 4 + 8))
+    assert splits >= 2 and ws == rows * splits * 128 * 4 + rows * splits * 8
+    assert api.decode_mq_workspace_size(full, 64, 17, 131072) == 0    # unsupported T
+    assert api.decode_mq_workspace_size(full, 64, 4, 3) == 0           # max_len < T
