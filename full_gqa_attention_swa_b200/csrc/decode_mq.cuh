@@ -15,10 +15,12 @@
 //
 // Work split: one CTA per (sequence, kv-head, split of the cache), as in the
 // one-query decode, but the M dimension of the m16n8k16 MMAs is now the
-// T * G (query, head) rows of the kv-head: consumer warp w owns rows
-// 16w .. 16w + 15 over every key of the split, so the warps never merge.  A
-// producer warp streams 32-key K/V stages with TMA; the last split also runs
-// one 16-key block of new tokens, staged by the consumers before the loop.
+// T * G (query, head) rows of the kv-head: warp w owns rows 16w .. 16w + 15
+// over every key of the split, so the warps never merge.  One elected thread
+// streams 32-key K/V stages with TMA (no producer warp: at 49 KB of stages and
+// at most 168 registers, four CTAs share an SM, so the 512 (sequence,
+// kv-head) pairs of a 64-sequence batch run in one wave); the last split also
+// runs one 16-key block of new tokens, staged into a free stage after the loop.
 // Cache bytes are still read once per (sequence, kv-head); the T-fold rows
 // raise the tensor work per byte, which stays far below the MMA rate.
 #pragma once
@@ -37,20 +39,18 @@ using decode_detail::mma_bf16;
 using decode_detail::sigmoidf_;
 using decode_detail::sw128_off;
 
-constexpr int kNewRows = 16;                       // new-token block (T <= 16), zero-padded
-constexpr uint32_t kNewBoxBytes = kNewRows * 128;  // one 64-dim half of the 16 rows
+constexpr int kNewRows = 16;  // new-token block (T <= 16), zero-padded, staged in stage 0
 constexpr int kStages = 3;
-// resident CTAs per SM: three (57 KB of shared memory each); four m-tiles
-// would spill at the register share of three, so they run two per SM
-constexpr int ctas_per_sm(int mt) { return mt <= 3 ? 3 : 2; }
+// resident CTAs per SM: four (49 KB of shared memory each); four m-tiles
+// would spill at the register share of four, so they run three per SM
+constexpr int ctas_per_sm(int mt) { return mt <= 3 ? 4 : 3; }
 static_assert(kNewRows == kDecodeMqMaxT, "one block holds every new token");
 static_assert(ctas_per_sm(3) == decode_mq_ctas_per_sm(48) && ctas_per_sm(4) == decode_mq_ctas_per_sm(64),
               "the split plan sees the kernel's occupancy");
-static_assert(kStageBytes % 1024 == 0 && kNewBoxBytes % 1024 == 0, "boxes stay 1024-byte aligned");
+static_assert(kStageBytes % 1024 == 0 && kNewRows <= KB, "stage boxes stay 1024-byte aligned and hold the new rows");
 
 struct MqSmem {
   uint8_t stage[kStages][kStageBytes];  // K lo, K hi, V lo, V hi boxes of 32 keys
-  uint8_t fresh[4][kNewBoxBytes];       // the new tokens' K lo, K hi, V lo, V hi (same swizzle)
   uint64_t full[kStages];
   uint64_t empty[kStages];
   int abort_flag;
@@ -157,9 +157,12 @@ __device__ __forceinline__ void mq_block(RowState& R, uint32_t kbase, uint32_t v
   }
 }
 
-// grid (max_splits, Hkv, B); MT consumer warps (16 rows each) + 1 producer warp.
+// grid (max_splits, Hkv, B); MT warps of 16 rows each.  Lane 0 of warp 0
+// also issues the TMA loads: the first kStages blocks up front, then at the
+// top of step t the block t - 1 + kStages into the stage every warp released
+// after step t - 1.
 template <int MT>
-__global__ void __launch_bounds__((MT + 1) * 32, ctas_per_sm(MT))
+__global__ void __launch_bounds__(MT * 32, ctas_per_sm(MT))
     decode_mq_kernel(const DecodeMqArgs a, const __grid_constant__ CUtensorMap k_map,
                      const __grid_constant__ CUtensorMap v_map) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -185,62 +188,35 @@ __global__ void __launch_bounds__((MT + 1) * 32, ctas_per_sm(MT))
   const int dead_slot = (ring && L0 >= a.window) ? (newest + 1) % a.window : -1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
+  const bool issuer = threadIdx.x == 0;
+  const int row3 = b * a.Hkv + kvh;
+  auto issue = [&](int t) {
+    const int s = t % kStages;
+    const int key0 = k_begin + t * KB;
+    uint8_t* st = sm.stage[s];
+    mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+    tma_load_3d(st, &k_map, &sm.full[s], 0, key0, row3);
+    tma_load_3d(st + kBoxBytes, &k_map, &sm.full[s], 64, key0, row3);
+    tma_load_3d(st + 2 * kBoxBytes, &v_map, &sm.full[s], 0, key0, row3);
+    tma_load_3d(st + 3 * kBoxBytes, &v_map, &sm.full[s], 64, key0, row3);
+  };
+  int issued = 0;
+  if (issuer) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], MT);
     }
     sm.abort_flag = 0;
     fence_mbar_init();
-  }
-  if (has_new && warp < MT) {
-    // the new tokens' K and V rows (zero past T) into the swizzled fresh boxes
-    for (int i = threadIdx.x; i < 2 * kNewRows * 16; i += MT * 32) {
-      const int tensor = i / (kNewRows * 16), row = (i >> 4) % kNewRows, ch = i & 15;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row < T) {
-        const uint16_t* src = (tensor ? a.v_new : a.k_new) + (((size_t)b * T + row) * a.Hkv + kvh) * kHeadDim;
-        v = __ldg(reinterpret_cast<const uint4*>(src) + ch);
-      }
-      *reinterpret_cast<uint4*>(sm.fresh[tensor * 2 + (ch >> 3)] + sw128_off(row, ch & 7)) = v;
+    if (n_blocks > 0) {
+      prefetch_tensormap(&k_map);
+      prefetch_tensormap(&v_map);
     }
+    for (; issued < n_blocks && issued < kStages; ++issued) issue(issued);
   }
   __syncthreads();
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == MT) {
-    // ------------------------------------------------------ TMA producer
-    if (lane == 0 && n_blocks > 0) {
-      prefetch_tensormap(&k_map);
-      prefetch_tensormap(&v_map);
-      const int row3 = b * a.Hkv + kvh;
-      int issued = 0;
-      for (int t = 0; t < n_blocks; ++t) {
-        const int s = t % kStages, u = t / kStages;
-        if (u > 0 && !mbar_wait(&sm.empty[s], (u - 1) & 1, abort_flag)) {
-          record_error(kErrDecodeMq + 1);
-          *abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
-        const int key0 = k_begin + t * KB;
-        uint8_t* st = sm.stage[s];
-        tma_load_3d(st, &k_map, &sm.full[s], 0, key0, row3);
-        tma_load_3d(st + kBoxBytes, &k_map, &sm.full[s], 64, key0, row3);
-        tma_load_3d(st + 2 * kBoxBytes, &v_map, &sm.full[s], 0, key0, row3);
-        tma_load_3d(st + 3 * kBoxBytes, &v_map, &sm.full[s], 64, key0, row3);
-        issued = t + 1;
-      }
-      if (*abort_flag) {
-        // let every copy this warp started land before the CTA exits
-        for (int t = issued > kStages ? issued - kStages : 0; t < issued; ++t)
-          mbar_wait(&sm.full[t % kStages], (t / kStages) & 1, nullptr, 200000000ull);
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
   const int g = lane >> 2, tig = lane & 3;
   const int G = a.G, n_rows = T * G;
   const int r0 = warp * 16 + g, r1 = r0 + 8;
@@ -271,7 +247,16 @@ __global__ void __launch_bounds__((MT + 1) * 32, ctas_per_sm(MT))
 
   for (int t = 0; t < n_blocks; ++t) {
     const int s = t % kStages;
-    if (!mbar_wait(&sm.full[s], (t / kStages) & 1, abort_flag)) {
+    if (issuer && t > 0 && issued < n_blocks) {
+      // every warp has released step t - 1's stage: refill it
+      if (!mbar_wait(&sm.empty[(t - 1) % kStages], ((t - 1) / kStages) & 1, abort_flag)) {
+        record_error(kErrDecodeMq + 1);
+        *abort_flag = 1;
+      } else {
+        issue(issued++);
+      }
+    }
+    if (*abort_flag || !mbar_wait(&sm.full[s], (t / kStages) & 1, abort_flag)) {
       record_error(kErrDecodeMq + 2);
       *abort_flag = 1;
       break;
@@ -305,15 +290,34 @@ __global__ void __launch_bounds__((MT + 1) * 32, ctas_per_sm(MT))
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[s]);
   }
-  if (*abort_flag) return;
+  __syncthreads();  // every warp is past the loop, aborted or not
+  if (*abort_flag) {
+    // let every copy the issuer started land before the CTA exits
+    if (issuer)
+      for (int t = issued > kStages ? issued - kStages : 0; t < issued; ++t)
+        mbar_wait(&sm.full[t % kStages], (t / kStages) & 1, nullptr, 200000000ull);
+    return;
+  }
 
   if (has_new) {
-    const uint32_t fb = smem_u32(sm.fresh[0]);
+    // every warp is past its last stage read and every load has landed:
+    // stage 0 takes the new tokens' K and V rows (zero past T)
+    for (int i = threadIdx.x; i < 2 * kNewRows * 16; i += MT * 32) {
+      const int tensor = i / (kNewRows * 16), row = (i >> 4) % kNewRows, ch = i & 15;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < T) {
+        const uint16_t* src = (tensor ? a.v_new : a.k_new) + (((size_t)b * T + row) * a.Hkv + kvh) * kHeadDim;
+        v = __ldg(reinterpret_cast<const uint4*>(src) + ch);
+      }
+      *reinterpret_cast<uint4*>(sm.stage[0] + (tensor * 2 + (ch >> 3)) * kBoxBytes + sw128_off(row, ch & 7)) = v;
+    }
+    __syncthreads();
+    const uint32_t fb = smem_u32(sm.stage[0]);
     auto vis = [&](int j, int hi) -> bool {
       const int tq = hi ? t1 : t0;
       return j <= tq && (!ring || j > tq - W);
     };
-    mq_block<kNewRows, true>(R, fb, fb + 2 * kNewBoxBytes, kNewBoxBytes, c, lane, kNewRows, -1, vis);
+    mq_block<kNewRows, true>(R, fb, fb + 2 * kBoxBytes, kBoxBytes, c, lane, kNewRows, -1, vis);
   }
 
   float l0 = R.l0, l1 = R.l1;
@@ -386,7 +390,7 @@ cudaError_t launch_mq(const DecodeMqArgs& a, const CUtensorMap& k_map, const CUt
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_mq_kernel<MT><<<dim3(a.max_splits, a.Hkv, a.B), (MT + 1) * 32, smem, stream>>>(a, k_map, v_map);
+  decode_mq_kernel<MT><<<dim3(a.max_splits, a.Hkv, a.B), MT * 32, smem, stream>>>(a, k_map, v_map);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.max_splits == 1) return e;
   decode_mq_combine_kernel<<<dim3(a.Hq, a.T, a.B), kHeadDim, 0, stream>>>(a);

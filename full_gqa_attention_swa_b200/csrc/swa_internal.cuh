@@ -126,7 +126,7 @@ constexpr int kDecodeKeyBlock = 32;   // keys per pipeline stage
 constexpr int kDecodeMqMaxT = 16;      // new tokens per sequence
 constexpr int kDecodeMqMaxRows = 64;   // T * G (query, head) rows per kv-head
 // resident multi-query decode CTAs per SM for T * G rows (sizes the split plan)
-constexpr int decode_mq_ctas_per_sm(int rows) { return rows <= 48 ? 3 : 2; }
+constexpr int decode_mq_ctas_per_sm(int rows) { return rows <= 48 ? 4 : 3; }
 
 struct DecodeMqArgs {
   int B, T, Hq, Hkv, G;
