@@ -75,19 +75,23 @@ __device__ __forceinline__ void mq_block(RowState& R, uint32_t kbase, uint32_t v
                                          int lane, int live, int dead, Vis vis) {
   constexpr int NT = NK / 8;
   const int tig = lane & 3;
+  // S: the NT accumulation chains advance together, one 32-dim step at a
+  // time, so NT independent MMAs are in flight behind each other
   float sc[NT][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-    const int krow = nt * 8 + (lane & 7);
+  for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < 8; kk += 2) {
-      const int ch = 2 * kk + (lane >> 3);  // 16-byte chunk (8 dims) 0..15
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(kbase + (ch >> 3) * box + sw128_off(krow, ch & 7), b0, b1, b2, b3);
-      mma_bf16(sc[nt], R.qf[kk], b0, b1);
-      mma_bf16(sc[nt], R.qf[kk + 1], b2, b3);
-    }
+  for (int kk = 0; kk < 8; kk += 2) {
+    const int ch = 2 * kk + (lane >> 3);  // 16-byte chunk (8 dims) 0..15
+    uint32_t kb[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      ldsm_x4(kbase + (ch >> 3) * box + sw128_off(nt * 8 + (lane & 7), ch & 7), kb[nt][0], kb[nt][1], kb[nt][2],
+              kb[nt][3]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], R.qf[kk], kb[nt][0], kb[nt][1]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], R.qf[kk + 1], kb[nt][2], kb[nt][3]);
   }
   float p[NT][4];
   float mx0 = -INFINITY, mx1 = -INFINITY;
