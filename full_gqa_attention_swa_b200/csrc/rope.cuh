@@ -189,6 +189,72 @@ __global__ void __launch_bounds__(256, 3) rope_kernel(const RopeArgs a) {
   }
 }
 
+// Keys only, into a separate buffer, no cache (the prefill pre-pass): the
+// same lanes and arithmetic as rope_kernel, but every load of the lane's
+// heads is issued before the cos/sin and the first store, so a thread waits
+// for DRAM once per group of kKeyGroup heads instead of once per head.  With
+// rotary_dim / 2 a multiple of 8, a chunk is wholly first half (role 1),
+// second half (role 2) or pass-through, and its partner is one whole chunk.
+constexpr int kKeyGroup = 4;
+
+__global__ void __launch_bounds__(256, 2) rope_keys_kernel(const RopeArgs a) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int chunk = (int)(tid & (kChunks - 1));
+  const long long tok = tid >> 4;
+  const long long n_tok = (long long)a.B * a.S;
+  const bool active = tok < n_tok;
+  const long long tk = active ? tok : 0;
+  const int b = (int)(tk / a.S);
+  const int s_idx = (int)(tk % a.S);
+  const int p = a.pos ? a.pos[tk] : a.pos0 + s_idx;
+  const int r = a.rotate ? a.rotary_dim : 0;
+  const int half = r / 2;
+  const int d0 = chunk * 8;
+  const int role = d0 < half ? 1 : (d0 < r ? 2 : 0);
+  const int k0 = role == 2 ? d0 - half : d0;                 // frequency index of element 0
+  const int pchunk = role == 1 ? chunk + half / 8 : chunk - half / 8;
+  const long long dst_tok = (long long)b * (a.dst_rows > 0 ? a.dst_rows : a.S) + a.dst_row_off + s_idx;
+  const int hs = blockIdx.y, nhs = gridDim.y;
+  bool first = true;
+  for (int h0 = hs; h0 < a.Hkv; h0 += nhs * kKeyGroup) {
+    uint4 own[kKeyGroup], par[kKeyGroup];
+#pragma unroll
+    for (int g = 0; g < kKeyGroup; ++g) {
+      const int h = h0 + g * nhs;
+      own[g] = par[g] = make_uint4(0u, 0u, 0u, 0u);
+      if (active && h < a.Hkv) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.k_src + (tk * a.Hkv + h) * kHeadDim);
+        own[g] = __ldg(src + chunk);
+        if (role != 0) par[g] = __ldg(src + pchunk);
+      }
+    }
+    float c[8], sn[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = 1.f;
+      sn[e] = 0.f;
+      if (role != 0) rope_cos_sin((double)p * a.inv_freq[k0 + e], &c[e], &sn[e]);
+    }
+    if (first && role == 1 && a.table && active && b == 0 && blockIdx.y == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a.table[rope_table_index(s_idx, k0 + e, half)] = make_float2(c[e], sn[e]);
+    }
+    first = false;
+    const float sgn = role == 1 ? -1.f : 1.f;  // y = x c - x' s (first half), x c + x' s (second)
+#pragma unroll
+    for (int g = 0; g < kKeyGroup; ++g) {
+      const int h = h0 + g * nhs;
+      if (!active || h >= a.Hkv) continue;
+      float x[8], xp[8], y[8];
+      unpack8(own[g], x);
+      unpack8(par[g], xp);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = role == 0 ? x[e] : x[e] * c[e] + sgn * (xp[e] * sn[e]);
+      *reinterpret_cast<uint4*>(a.k_dst + (dst_tok * a.Hkv + h) * kHeadDim + chunk * 8) = pack8(y);
+    }
+  }
+}
+
 }  // namespace rope_detail
 
 cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
@@ -203,7 +269,12 @@ cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
   while (blocks * hsplit < 148 * 4 && hsplit < max_heads) hsplit *= 2;
   if (hsplit > max_heads) hsplit = max_heads;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  rope_detail::rope_kernel<<<dim3((unsigned)blocks, (unsigned)hsplit), threads, 0, stream>>>(a);
+  const int r = a.rotate ? a.rotary_dim : 0;
+  const bool keys_only = !a.q && a.k_src && !a.k_cache && a.k_dst != a.k_src && ((r / 2) % 8) == 0;
+  if (keys_only)
+    rope_detail::rope_keys_kernel<<<dim3((unsigned)blocks, (unsigned)hsplit), threads, 0, stream>>>(a);
+  else
+    rope_detail::rope_kernel<<<dim3((unsigned)blocks, (unsigned)hsplit), threads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
