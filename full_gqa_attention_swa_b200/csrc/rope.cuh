@@ -108,14 +108,16 @@ __device__ __forceinline__ void rotate_chunk(const uint16_t* row_src, uint16_t* 
 // fp64 and reduced to [-pi, pi] by subtracting the nearest multiple of 2*pi
 // (Cody-Waite reduction with 2*pi split into a double and its rounding
 // remainder), so its error stays near 1e-15 rad for any position below 2^31;
-// the reduced angle is then rounded to fp32 for sincosf.
+// the reduced angle is then rounded to fp32 for the hardware sine / cosine
+// (__sincosf: absolute error below 1e-6 on [-pi, pi], far under the bf16
+// rounding of every rotated value).
 __device__ __forceinline__ void rope_cos_sin(double angle, float* c, float* s) {
   const double kTwoPiHi = 6.283185307179586;       // 2*pi rounded to double
   const double kTwoPiLo = 2.4492935982947064e-16;  // 2*pi - kTwoPiHi
   const double n = rint(angle * (1.0 / kTwoPiHi));
   double r = fma(-n, kTwoPiHi, angle);
   r = fma(-n, kTwoPiLo, r);
-  sincosf((float)r, s, c);
+  __sincosf((float)r, s, c);
 }
 
 // grid.x: ceil(B*S*16 / blockDim.x); grid.y: head split (heads h with
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(256, 3) rope_kernel(const RopeArgs a) {
 // for DRAM once per group of kKeyGroup heads instead of once per head.  With
 // rotary_dim / 2 a multiple of 8, a chunk is wholly first half (role 1),
 // second half (role 2) or pass-through, and its partner is one whole chunk.
-constexpr int kKeyGroup = 4;
+constexpr int kKeyGroup = 8;
 
 __global__ void __launch_bounds__(256, 2) rope_keys_kernel(const RopeArgs a) {
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -271,8 +273,12 @@ cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   const int r = a.rotate ? a.rotary_dim : 0;
   const bool keys_only = !a.q && a.k_src && !a.k_cache && a.k_dst != a.k_src && ((r / 2) % 8) == 0;
-  if (keys_only)
-    rope_detail::rope_keys_kernel<<<dim3((unsigned)blocks, (unsigned)hsplit), threads, 0, stream>>>(a);
+  if (keys_only) {
+    // one head split while a lane's heads fit one load group: each split
+    // recomputes the lane's cos/sin
+    const unsigned ks = (unsigned)(a.Hkv <= rope_detail::kKeyGroup ? 1 : hsplit);
+    rope_detail::rope_keys_kernel<<<dim3((unsigned)blocks, ks), threads, 0, stream>>>(a);
+  }
   else
     rope_detail::rope_kernel<<<dim3((unsigned)blocks, (unsigned)hsplit), threads, 0, stream>>>(a);
   return cudaGetLastError();
