@@ -151,3 +151,27 @@ def test_persistent_multi_tile(cuda_device, Hq, Hkv, W, B):
     got = out.cpu()[torch.from_numpy(rows[:, 0]), torch.from_numpy(rows[:, 1]), torch.from_numpy(rows[:, 2])]
     assert_close(got, ref, f"multi-tile Hq{Hq} Hkv{Hkv} W{W} B{B}")
     check_no_device_error()
+
+
+@pytest.mark.slow
+def test_q_and_out_beyond_2_31_elements(cuda_device):
+    """Maximum-size indexing: B2 S69632 Hq128 puts 2^31 + 2^27 elements in q
+    and out (4.6 GB each), so every 64-bit offset (rows, gate, cos/sin table,
+    output) is exercised; a W64 band keeps the work small.  Sampled rows
+    include the last rows of the second sequence."""
+    B, S, Hq, Hkv, W = 2, 69632, 128, 8, 64
+    assert B * S * Hq * 128 > 2 ** 31
+    p = api.LayerParams(Hq, Hkv, 128, W, 5e5, 128)
+    d = inputs.prefill_inputs(B, S, Hq, Hkv, 128, seed=760, device=cuda_device)
+    out = api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"])
+    torch.cuda.synchronize()
+    rows = prefill_rows_sample(B, S, Hq, W, 760, n_random=96)
+    rows = np.concatenate([rows, np.array([(1, S - 1, Hq - 1), (1, S - 1, 0), (1, S - 129, 77)], np.int64)])
+    got = out[torch.from_numpy(rows[:, 0]).to(cuda_device), torch.from_numpy(rows[:, 1]).to(cuda_device),
+              torch.from_numpy(rows[:, 2]).to(cuda_device)].cpu()
+    del out
+    q = bits(d["q"].cpu())
+    ref = oracle.prefill(oracle_layer(p), q, bits(d["k"].cpu()), bits(d["v"].cpu()), d["gate"].cpu().numpy(),
+                         rows=rows)
+    assert_close(got, ref, "q/out beyond 2^31 elements")
+    check_no_device_error()
