@@ -291,36 +291,60 @@ def bench_prefill_chunk(c, steps: int, warmup: int, dev):
 
 
 def bench_prefill_e2e(c, steps: int, dev):
-    """Same metric through the public API with host buffers: pinned host
-    inputs copied in and the output copied back every step."""
+    """Same metric through the public API with host buffers: every step copies
+    its pinned host inputs in and its output back.  Steps are pipelined as a
+    serving loop would run them: two device buffer sets, the next step's
+    host->device copy on one stream, attention on the current stream, the
+    device->host copy of the result on a third (the link is full duplex)."""
     from full_gqa_attention_swa_b200 import api
 
     p = _layer(c)
     host = inputs.prefill_inputs(c.B, c.S, c.Hq, c.Hkv, 128, c.seed)
     host = {k: t.pin_memory() for k, t in host.items()}
     out_host = torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16).pin_memory()
-    d = {k: torch.empty_like(t, device=dev) for k, t in host.items()}
-    out = torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16, device=dev)
+    bufs = [{k: torch.empty_like(t, device=dev) for k, t in host.items()} for _ in range(2)]
+    outs = [torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     ws = torch.empty(max(api.prefill_workspace_size(p, c.B, c.S), 1), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    comp = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]   # attention on buffer b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # output of buffer b copied back
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
+    n = [0]
 
     def step():
-        for k in d:
-            d[k].copy_(host[k], non_blocking=True)
-        api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"], out=out, workspace=ws, stream=stream)
-        out_host.copy_(out, non_blocking=True)
+        b = n[0] % 2
+        if n[0] >= 2:
+            s_in.wait_event(ev_done[b])        # attention of two steps ago no longer reads bufs[b]
+        with torch.cuda.stream(s_in):
+            for k in host:
+                bufs[b][k].copy_(host[k], non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        if n[0] >= 2:
+            comp.wait_event(ev_out[b])         # outs[b] of two steps ago has been read back
+        d = bufs[b]
+        api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"], out=outs[b], workspace=ws, stream=comp)
+        ev_done[b].record(comp)
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            out_host.copy_(outs[b], non_blocking=True)
+            ev_out[b].record(s_out)
+        n[0] += 1
 
     for _ in range(2):
         step()
     torch.cuda.synchronize(dev)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
+    ev0.record(comp)
+    s_in.wait_event(ev0)
     for _ in range(steps):
         step()
-    ev1.record(stream)
+    comp.wait_event(ev_out[(n[0] - 1) % 2])    # the last result is on the host
+    ev1.record(comp)
     torch.cuda.synchronize(dev)
     return ev0.elapsed_time(ev1), h2d, d2h
 
