@@ -98,7 +98,7 @@ PREFILL_TRAFFIC = {
     "workload": "step37_sliding_B1_S8192_Hq96_Hkv8_W512",
     "bytes": 402.3e6,
     # prefill.cuh and ptx.cuh (the kernel and its PTX helpers) as captured; any change makes the figure stale
-    "source_sha256": "9767bf0b33fa98554812f667b18acbdbda37877106df8376d0bfc2ceaa139514",
+    "source_sha256": "d4566b0dd4deca3c3ea5079d21dad10e4756b31362501c4283f8a5613b40fb4d",
 }
 PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh")
 

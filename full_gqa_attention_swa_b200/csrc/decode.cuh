@@ -346,16 +346,14 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& k_map, const C
   if (a.B == 0) return cudaSuccess;
   using namespace decode_detail;
   const size_t smem = sizeof(DecodeSmem<kStages>) + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static DeviceOnce setup;
+  cudaError_t e = device_once(setup, [&](int, int*) {
+    return cudaFuncSetAttribute(decode_split_kernel<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid(a.max_splits, a.Hkv, a.B);
   decode_split_kernel<kStages><<<grid, kThreads, smem, stream>>>(a, k_map, v_map);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess || a.max_splits == 1) return e;
   decode_combine_kernel<<<dim3(a.Hq, a.B), kHeadDim, 0, stream>>>(a);
   return cudaGetLastError();

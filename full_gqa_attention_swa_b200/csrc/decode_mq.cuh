@@ -387,15 +387,13 @@ template <int MT>
 cudaError_t launch_mq(const DecodeMqArgs& a, const CUtensorMap& k_map, const CUtensorMap& v_map,
                       cudaStream_t stream) {
   const size_t smem = sizeof(MqSmem) + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mq_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static DeviceOnce setup;
+  cudaError_t e = device_once(setup, [&](int, int*) {
+    return cudaFuncSetAttribute(decode_mq_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
+  if (e != cudaSuccess) return e;
   decode_mq_kernel<MT><<<dim3(a.max_splits, a.Hkv, a.B), MT * 32, smem, stream>>>(a, k_map, v_map);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess || a.max_splits == 1) return e;
   decode_mq_combine_kernel<<<dim3(a.Hq, a.T, a.B), kHeadDim, 0, stream>>>(a);
   return cudaGetLastError();

@@ -779,25 +779,21 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& q_map, con
   if (n_tiles == 0) return cudaSuccess;
   if (n_tiles > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   const size_t smem = sizeof(PrefillSmem);
-  static int n_sm = 0;
-  static bool checked = false;
-  if (!checked) {
-    cudaError_t e =
+  static DeviceOnce setup;
+  int n_sm = 0;
+  cudaError_t e = device_once(setup, [&](int dev, int* sm_count) -> cudaError_t {
+    cudaError_t r =
         cudaFuncSetAttribute(prefill_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if (r != cudaSuccess) return r;
     // setmaxnreg redistributes the registers the CTA was launched with: the
     // kernel must be launched with exactly kRegsLaunch per thread
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, prefill_kernel<kMode>);
-    if (e != cudaSuccess) return e;
+    r = cudaFuncGetAttributes(&fa, prefill_kernel<kMode>);
+    if (r != cudaSuccess) return r;
     if (fa.numRegs != (int)kRegsLaunch) return cudaErrorInvalidConfiguration;
-    int dev = 0;
-    e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    checked = true;
-  }
+    return cudaDeviceGetAttribute(sm_count, cudaDevAttrMultiProcessorCount, dev);
+  }, &n_sm);
+  if (e != cudaSuccess) return e;
   const int grid = (int)(n_tiles < n_sm ? n_tiles : n_sm);
   prefill_kernel<kMode><<<grid, kThreads, smem, stream>>>(a, q_map, k_map, v_map, o_map);
   return cudaGetLastError();

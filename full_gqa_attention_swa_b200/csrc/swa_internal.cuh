@@ -6,9 +6,38 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "ptx.cuh"
 
 namespace swa {
+
+// One-time setup per device for a launcher: kernel attributes (the opt-in
+// shared memory size) belong to a device context, so a process that drives
+// several GPUs sets them on each.  fn(dev, &value) runs once per device
+// ordinal, under a lock; value (e.g. the SM count) is returned every call.
+constexpr int kMaxSetupDevices = 64;
+struct DeviceOnce {
+  std::mutex mu;
+  uint64_t done = 0;
+  int value[kMaxSetupDevices] = {};
+};
+
+template <class Fn>
+cudaError_t device_once(DeviceOnce& o, Fn fn, int* value_out = nullptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSetupDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(o.mu);
+  if (!((o.done >> dev) & 1ull)) {
+    e = fn(dev, &o.value[dev]);
+    if (e != cudaSuccess) return e;
+    o.done |= 1ull << dev;
+  }
+  if (value_out) *value_out = o.value[dev];
+  return cudaSuccess;
+}
 
 constexpr int kHeadDim = 128;
 constexpr int kMaxRotaryHalf = kHeadDim / 2;
