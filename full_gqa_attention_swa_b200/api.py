@@ -159,6 +159,20 @@ def _need(t, name, dtype, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _device(*tensors, stream=None):
+    """The one CUDA device every given tensor lives on.  The call runs with
+    it current (and on its current stream unless one is given): the library
+    takes plain pointers, and a pointer into another GPU's memory would reach
+    a kernel as an invalid address."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"tensors must all be on one CUDA device, got {sorted(str(d) for d in devs)}")
+    dev = devs.pop()
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, tensors on {dev}")
+    return dev
+
+
 def version() -> str:
     return load().swa_version().decode()
 
@@ -186,8 +200,9 @@ def rope_qk(layer: LayerParams, q=None, k=None, pos=None, pos0: int = 0, v=None,
         C = k_cache.shape[2]
         _need(k_cache, "k_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
         _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
-    _check(load().swa_rope_qk(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(pos), int(pos0), _ptr(v),
-                              _ptr(k_cache), _ptr(v_cache), C, _stream(stream)))
+    with torch.cuda.device(_device(q, k, pos, v, k_cache, v_cache, stream=stream)):
+        _check(load().swa_rope_qk(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(pos), int(pos0), _ptr(v),
+                                  _ptr(k_cache), _ptr(v_cache), C, _stream(stream)))
 
 
 def prefill_workspace_size(layer: LayerParams, B: int, S: int) -> int:
@@ -210,8 +225,9 @@ def attn_prefill(layer: LayerParams, q, k, v, gate=None, out=None, workspace=Non
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load().swa_attn_prefill(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(v), _ptr(gate),
-                                   _ptr(out), _ptr(workspace), nbytes, _stream(stream)))
+    with torch.cuda.device(_device(q, k, v, gate, out, workspace, stream=stream)):
+        _check(load().swa_attn_prefill(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(v), _ptr(gate),
+                                       _ptr(out), _ptr(workspace), nbytes, _stream(stream)))
     return out
 
 
@@ -241,9 +257,10 @@ def attn_prefill_chunk(layer: LayerParams, pos0: int, q, k, v, gate, k_cache, v_
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load().swa_attn_prefill_chunk(ctypes.byref(layer.c()), B, S, int(pos0), _ptr(q), _ptr(k), _ptr(v),
-                                         _ptr(gate), _ptr(k_cache), _ptr(v_cache), C, _ptr(out), _ptr(workspace),
-                                         nbytes, _stream(stream)))
+    with torch.cuda.device(_device(q, k, v, gate, k_cache, v_cache, out, workspace, stream=stream)):
+        _check(load().swa_attn_prefill_chunk(ctypes.byref(layer.c()), B, S, int(pos0), _ptr(q), _ptr(k), _ptr(v),
+                                             _ptr(gate), _ptr(k_cache), _ptr(v_cache), C, _ptr(out), _ptr(workspace),
+                                             nbytes, _stream(stream)))
     return out
 
 
@@ -271,9 +288,10 @@ def attn_decode(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens, max_len
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load().swa_attn_decode(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache), _ptr(v_cache), C,
-                                  _ptr(seq_lens), int(max_len), _ptr(out), _ptr(workspace), nbytes,
-                                  _stream(stream)))
+    with torch.cuda.device(_device(q, gate, k_cache, v_cache, seq_lens, out, workspace, stream=stream)):
+        _check(load().swa_attn_decode(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache), _ptr(v_cache), C,
+                                      _ptr(seq_lens), int(max_len), _ptr(out), _ptr(workspace), nbytes,
+                                      _stream(stream)))
     return out
 
 
@@ -304,9 +322,10 @@ def attn_decode_mq(layer: LayerParams, q, gate, k_new, v_new, k_cache, v_cache, 
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load().swa_attn_decode_mq(ctypes.byref(layer.c()), B, T, _ptr(q), _ptr(gate), _ptr(k_new), _ptr(v_new),
-                                     _ptr(k_cache), _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
-                                     _ptr(workspace), nbytes, _stream(stream)))
+    with torch.cuda.device(_device(q, gate, k_new, v_new, k_cache, v_cache, seq_lens, out, workspace, stream=stream)):
+        _check(load().swa_attn_decode_mq(ctypes.byref(layer.c()), B, T, _ptr(q), _ptr(gate), _ptr(k_new), _ptr(v_new),
+                                         _ptr(k_cache), _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
+                                         _ptr(workspace), nbytes, _stream(stream)))
     return out
 
 
@@ -326,9 +345,10 @@ def attn_decode_no_alloc(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens
     _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
     _need(seq_lens, "seq_lens", torch.int32, (B,))
     _need(out, "out", torch.bfloat16, (B, layer.num_q_heads, D))
-    _check(load().swa_attn_decode_no_alloc(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache),
-                                           _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
-                                           _stream(stream)))
+    with torch.cuda.device(_device(q, gate, k_cache, v_cache, seq_lens, out, stream=stream)):
+        _check(load().swa_attn_decode_no_alloc(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache),
+                                               _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
+                                               _stream(stream)))
     return out
 
 

@@ -26,7 +26,9 @@
  * Conventions for every call:
  *   - Tensors are device pointers to contiguous row-major arrays in the layout
  *     stated at each argument; bf16 tensors are passed as uint16_t (their bit
- *     patterns).  Every tensor pointer must be 16-byte aligned.
+ *     patterns).  Every tensor pointer must be 16-byte aligned and point into
+ *     the memory of the current device (the one `stream` belongs to); the
+ *     calls do not check the device of a pointer.
  *   - The caller owns all memory.  No call allocates device memory; calls that
  *     need scratch take a caller-provided workspace whose size a *_size()
  *     query returns.

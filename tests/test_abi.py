@@ -237,3 +237,19 @@ def test_decode_mq_workspace_sizes(lib):
     assert splits >= 2 and ws == rows * splits * 128 * 4 + rows * splits * 8
     assert api.decode_mq_workspace_size(full, 64, 17, 131072) == 0    # unsupported T
     assert api.decode_mq_workspace_size(full, 64, 4, 3) == 0           # max_len < T
+
+
+def test_binding_requires_one_device():
+    """The binding refuses tensors spread over several GPUs (a pointer into
+    another GPU's memory must never reach a kernel) and a stream of another
+    device; no GPU is needed to check the rule."""
+    from types import SimpleNamespace as NS
+
+    import torch
+
+    d0, d1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    assert api._device(NS(device=d0), None, NS(device=d0)) == d0
+    with pytest.raises(ValueError):
+        api._device(NS(device=d0), NS(device=d1))
+    with pytest.raises(ValueError):
+        api._device(NS(device=d1), stream=NS(device=d0))
