@@ -95,8 +95,9 @@ __device__ __forceinline__ void rotate_chunk(const uint16_t* row_src, uint16_t* 
     float x[8], y[8];
     unpack8(own, x);
     for (int e = 0; e < 8; ++e) {
-      if (L.role[e] == 1) y[e] = x[e] * c[e] - xp[e] * s[e];
-      else if (L.role[e] == 2) y[e] = x[e] * c[e] + xp[e] * s[e];
+      // one rounding order for every RoPE site: x c + (-/+ x' s), the product x' s rounded first
+      if (L.role[e] == 1) y[e] = fmaf(x[e], c[e], -(xp[e] * s[e]));
+      else if (L.role[e] == 2) y[e] = fmaf(x[e], c[e], xp[e] * s[e]);
       else y[e] = x[e];
     }
     *reinterpret_cast<uint4*>(row_dst + chunk * 8) = pack8(y);
@@ -191,8 +192,9 @@ __global__ void __launch_bounds__(256, 3) rope_kernel(const RopeArgs a) {
   }
 }
 
-// Keys only, into a separate buffer, no cache (the prefill pre-pass): the
-// same lanes and arithmetic as rope_kernel, but every load of the lane's
+// Keys into a separate buffer, optionally appended with the values to the KV
+// cache (the prefill pre-pass, a continued-prefill chunk): the same lanes,
+// arithmetic and slot rules as rope_kernel, but every load of the lane's
 // heads is issued before the cos/sin and the first store, so a thread waits
 // for DRAM once per group of kKeyGroup heads instead of once per head.  With
 // rotary_dim / 2 a multiple of 8, a chunk is wholly first half (role 1),
@@ -217,6 +219,16 @@ __global__ void __launch_bounds__(256, 2) rope_keys_kernel(const RopeArgs a) {
   const int pchunk = role == 1 ? chunk + half / 8 : chunk - half / 8;
   const long long dst_tok = (long long)b * (a.dst_rows > 0 ? a.dst_rows : a.S) + a.dst_row_off + s_idx;
   const int hs = blockIdx.y, nhs = gridDim.y;
+  // cache slot of this token: p mod W on a ring, p on a linear cache
+  long long slot = 0;
+  bool cache_it = false;
+  if (a.k_cache) {
+    slot = a.window > 0 ? (long long)(p % a.window) : (long long)p;
+    const bool fits = p >= 0 && slot < a.cache_capacity;
+    if (active && !fits && chunk == 0 && hs == 0) record_error(kErrRope + 1);
+    // consecutive positions on a ring: only the call's last W are kept
+    cache_it = active && fits && !(a.window > 0 && !a.pos && p <= a.pos0 + a.S - 1 - a.window);
+  }
   bool first = true;
   for (int h0 = hs; h0 < a.Hkv; h0 += nhs * kKeyGroup) {
     uint4 own[kKeyGroup], par[kKeyGroup];
@@ -243,6 +255,7 @@ __global__ void __launch_bounds__(256, 2) rope_keys_kernel(const RopeArgs a) {
     }
     first = false;
     const float sgn = role == 1 ? -1.f : 1.f;  // y = x c - x' s (first half), x c + x' s (second)
+    // (the same rounding order as rope_kernel: the product x' s rounded, then one fma)
 #pragma unroll
     for (int g = 0; g < kKeyGroup; ++g) {
       const int h = h0 + g * nhs;
@@ -251,8 +264,28 @@ __global__ void __launch_bounds__(256, 2) rope_keys_kernel(const RopeArgs a) {
       unpack8(own[g], x);
       unpack8(par[g], xp);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = role == 0 ? x[e] : x[e] * c[e] + sgn * (xp[e] * sn[e]);
-      *reinterpret_cast<uint4*>(a.k_dst + (dst_tok * a.Hkv + h) * kHeadDim + chunk * 8) = pack8(y);
+      for (int e = 0; e < 8; ++e) y[e] = role == 0 ? x[e] : fmaf(x[e], c[e], sgn * (xp[e] * sn[e]));
+      const uint4 yk = pack8(y);
+      *reinterpret_cast<uint4*>(a.k_dst + (dst_tok * a.Hkv + h) * kHeadDim + chunk * 8) = yk;
+      if (cache_it)
+        *reinterpret_cast<uint4*>(a.k_cache + (((long long)b * a.Hkv + h) * a.cache_capacity + slot) * kHeadDim +
+                                  chunk * 8) = yk;
+    }
+    if (cache_it) {  // the raw values follow their keys into the cache
+      uint4 vv[kKeyGroup];
+#pragma unroll
+      for (int g = 0; g < kKeyGroup; ++g) {
+        const int h = h0 + g * nhs;
+        vv[g] = h < a.Hkv ? __ldg(reinterpret_cast<const uint4*>(a.v + (tk * a.Hkv + h) * kHeadDim) + chunk)
+                          : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int g = 0; g < kKeyGroup; ++g) {
+        const int h = h0 + g * nhs;
+        if (h < a.Hkv)
+          *reinterpret_cast<uint4*>(a.v_cache + (((long long)b * a.Hkv + h) * a.cache_capacity + slot) * kHeadDim +
+                                    chunk * 8) = vv[g];
+      }
     }
   }
 }
@@ -272,7 +305,7 @@ cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
   if (hsplit > max_heads) hsplit = max_heads;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   const int r = a.rotate ? a.rotary_dim : 0;
-  const bool keys_only = !a.q && a.k_src && !a.k_cache && a.k_dst != a.k_src && ((r / 2) % 8) == 0;
+  const bool keys_only = !a.q && a.k_src && a.k_dst != a.k_src && ((r / 2) % 8) == 0;
   if (keys_only) {
     // one head split while a lane's heads fit one load group: each split
     // recomputes the lane's cos/sin
