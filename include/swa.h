@@ -119,9 +119,8 @@ SWA_API swa_status swa_rope_qk(const swa_layer_params* params, int32_t B, int32_
  * swa_prefill_workspace_size -- bytes of workspace swa_attn_prefill needs for
  * (params, B, S): the rotated keys [B, S, Hkv, D] bf16 plus the fp32 cos/sin
  * table of positions 0..S-1 (rounded up to a multiple of 32 positions), each
- * 256-byte aligned; 0 when the layer applies
- * no rotary encoding.  Returns 0 for invalid
- * parameters.
+ * 256-byte aligned; 0 when the layer applies no rotary encoding.  Returns 0
+ * for invalid parameters.
  */
 SWA_API size_t swa_prefill_workspace_size(const swa_layer_params* params, int32_t B, int32_t S);
 
