@@ -574,13 +574,19 @@ def main():
                         "frac": achieved / peaks["bf16_tflops"], "traffic": measured_prefill_traffic(c.name),
                         "peak_source": f"{peak_src} bf16 burst",
                         "kernel": "swa_attn_prefill (key-RoPE pre-pass + attention kernel), CUDA events"}
-    if rank == 0 and not args.no_e2e:
+    if not args.no_e2e:
+        # every rank runs its own end-to-end loop at the same time (they share
+        # the host's links); the slowest rank's time counts
         e2e_steps = max(3, min(args.steps, 30))
+        if dist is not None:
+            dist.barrier()
         e_ms, h2d, d2h = bench_prefill_e2e(c, e2e_steps, dev)
-        line["e2e"] = {"value": flops * e2e_steps / (e_ms / 1e3) / 1e12 * world, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e_ms, dist, dev)
+        line["e2e"] = {"value": flops * e2e_steps * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     if rank == 0:
-        if not args.no_decode and args.only == "all":
+        # the extra legs and the CPU baseline describe one GPU: single-process runs only
+        if world == 1 and not args.no_decode and args.only == "all":
             extra = {}
             for dc in (configs.DECODE_SLIDING, configs.DECODE_FULL):
                 steps = 200 if dc.window > 0 else 10
@@ -603,7 +609,7 @@ def main():
                 chunks[cc.name] = {"ms": c_ms, "TFLOP/s": tf, "frac_bf16": tf / peaks["bf16_tflops"],
                                    "peak_source": f"{peak_src} bf16 burst"}
             line["prefill_chunk"] = chunks
-        if args.cpu_budget > 0:
+        if world == 1 and args.cpu_budget > 0:
             r, n, dt, thr = oracle_sample_rate(c, args.cpu_budget)
             line["cpu_baseline"] = {"value": r, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                     "sample": f"{n} seeded random (b, i, h) rows of {c.name}, {dt:.1f} s"}
