@@ -587,27 +587,24 @@ def main():
     if rank == 0:
         # the extra legs and the CPU baseline describe one GPU: single-process runs only
         if world == 1 and not args.no_decode and args.only == "all":
-            extra = {}
-            for dc in (configs.DECODE_SLIDING, configs.DECODE_FULL):
-                steps = 200 if dc.window > 0 else 10
-                d_ms, nbytes = bench_decode(dc, steps, 3, dev)
-                gbs = nbytes / (d_ms / 1e3) / 1e9
-                extra[dc.name] = {"ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
-                                  "peak_source": f"{peak_src} hbm copy"}
-            line["decode"] = extra
-            mqs = {}
-            for mc in (configs.MQ_SLIDING, configs.MQ_FULL):
-                d_ms, nbytes = bench_decode_mq(mc, 200 if mc.window > 0 else 10, 3, dev)
-                gbs = nbytes / (d_ms / 1e3) / 1e9
-                mqs[mc.name] = {"ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
-                                "peak_source": f"{peak_src} hbm copy"}
-            line["decode_mq"] = mqs
+            # the short legs first, the two 34 GB full-layer decode legs last
             chunks = {}
             for cc in (configs.CHUNK_SLIDING, configs.CHUNK_FULL):
                 c_ms = bench_prefill_chunk(cc, 20 if cc.window > 0 else 5, 3, dev)
                 tf = chunk_flops(cc) / (c_ms / 1e3) / 1e12
                 chunks[cc.name] = {"ms": c_ms, "TFLOP/s": tf, "frac_bf16": tf / peaks["bf16_tflops"],
                                    "peak_source": f"{peak_src} bf16 burst"}
+            extra, mqs = {}, {}
+            for kind, dc in (("decode", configs.DECODE_SLIDING), ("mq", configs.MQ_SLIDING),
+                             ("decode", configs.DECODE_FULL), ("mq", configs.MQ_FULL)):
+                steps = 200 if dc.window > 0 else 10
+                d_ms, nbytes = (bench_decode if kind == "decode" else bench_decode_mq)(dc, steps, 3, dev)
+                gbs = nbytes / (d_ms / 1e3) / 1e9
+                (extra if kind == "decode" else mqs)[dc.name] = {
+                    "ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                    "peak_source": f"{peak_src} hbm copy"}
+            line["decode"] = extra
+            line["decode_mq"] = mqs
             line["prefill_chunk"] = chunks
         if world == 1 and args.cpu_budget > 0:
             r, n, dt, thr = oracle_sample_rate(c, args.cpu_budget)
