@@ -572,7 +572,7 @@ swa_status swa_attn_decode(const swa_layer_params* p, int32_t B, const uint16_t*
   if (max_len < 1) return fail(SWA_ERR_INVALID_ARG, "max_len=%d must be >= 1", max_len);
   if (p->window < 0 && max_len > cache_capacity)
     return fail(SWA_ERR_INVALID_ARG, "full layer: max_len=%d exceeds cache_capacity=%d", max_len, cache_capacity);
-  if ((long long)B * Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B*Hkv=%lld too large", (long long)B * Hkv);
+  if (B > 65535 || Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B=%d or Hkv=%d too large (grid y / z)", B, Hkv);
   const DecodePlan pl = plan_decode(p, B, max_len);
   if (pl.total > 0) {
     if (!workspace) return fail(SWA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", pl.total);
@@ -671,7 +671,7 @@ swa_status swa_attn_decode_no_alloc(const swa_layer_params* p, int32_t B, const 
   if (max_len < 1) return fail(SWA_ERR_INVALID_ARG, "max_len=%d must be >= 1", max_len);
   if (p->window < 0 && max_len > cache_capacity)
     return fail(SWA_ERR_INVALID_ARG, "full layer: max_len=%d exceeds cache_capacity=%d", max_len, cache_capacity);
-  if ((long long)B * Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B*Hkv=%lld too large", (long long)B * Hkv);
+  if (B > 65535 || Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B=%d or Hkv=%d too large (grid y / z)", B, Hkv);
   DecodePlan pl;
   if ((st = plan_decode_no_alloc(p, B, max_len, &pl)) != SWA_OK) return st;
   void* scratch = nullptr;

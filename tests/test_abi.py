@@ -130,6 +130,7 @@ def test_decode_argument_errors(lib):
     a[8] = NULL                                                         # workspace missing
     assert lib.swa_attn_decode(full, 64, *a) == 3
     assert lib.swa_attn_decode(sl, 0, *args(512, 512)) == 0              # empty batch
+    assert lib.swa_attn_decode(sl, 70000, *args(512, 512)) == 2          # B beyond the grid's z limit
 
 
 def test_rope_argument_errors(lib):

@@ -134,3 +134,21 @@ def test_full_size_decode_sampled(cuda_device, cfg):
     got = out.cpu()[torch.from_numpy(rows[:, 0]), torch.from_numpy(rows[:, 1])]
     assert_close(got, ref, cfg.name)
     check_no_device_error()
+
+
+@pytest.mark.slow
+def test_large_batch(cuda_device):
+    """B = 9000 sequences (72000 (sequence, kv-head) pairs: the batch sits on
+    the grid's z axis), ring of 64; sampled sequences against the oracle."""
+    B, Hq, Hkv, W = 9000, 16, 8, 64
+    p = api.LayerParams(Hq, Hkv, 128, W, 1e4, 128)
+    lens = inputs.uniform_int(B, 1, 200, 4242)
+    d = inputs.decode_inputs(B, Hq, Hkv, 128, W, 4242, device=cuda_device)
+    out = api.attn_decode(p, d["q"], d["gate"], d["k_cache"], d["v_cache"], lens.to(cuda_device), 200)
+    torch.cuda.synchronize()
+    bsel = [0, 1, 4095, 4096, 8191, 8192, 8999]
+    sub = torch.tensor(bsel)
+    ref = oracle.decode(oracle_layer(p), oracle.bf16_bits_to_f64(bits(d["q"][sub].cpu())), d["gate"][sub].cpu().numpy(),
+                        bits(d["k_cache"][sub].cpu()), bits(d["v_cache"][sub].cpu()), lens[sub].numpy())
+    assert_close(out[sub.to(cuda_device)], ref, "decode B9000")
+    check_no_device_error()
