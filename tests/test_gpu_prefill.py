@@ -36,7 +36,7 @@ def test_tiny_config_all_rows(cuda_device):
 
 
 @pytest.mark.parametrize("W", [1, 2, 63, 64, 65, 127, 128, 129, 300, -1])
-@pytest.mark.parametrize("Hq", [4, 8])  # G = 2: single-SM kernel; G = 4: CTA-pair kernel
+@pytest.mark.parametrize("Hq", [4, 8])  # G = 2: one head pair per tile; G = 4: two pairs per (q-tile, kv-head)
 def test_window_sweep(cuda_device, W, Hq):
     p = api.LayerParams(Hq, 2, 128, W, 1e4, 128)
     _check_all_rows(cuda_device, p, 1, 300, seed=100 + max(W, 0))
@@ -138,7 +138,7 @@ def test_full_size_sampled_rows(cuda_device, cfg):
 @pytest.mark.parametrize("Hq,Hkv,W,B", [(16, 2, 512, 4), (16, 2, -1, 4), (4, 2, 300, 8), (12, 1, 200, 8)],
                          ids=["pair-sliding", "pair-causal", "single-sliding", "pair-G12"])
 def test_persistent_multi_tile(cuda_device, Hq, Hkv, W, B):
-    """More work tiles than CTAs (or CTA pairs): every CTA runs several tiles
+    """More work tiles than CTAs: every persistent CTA runs several tiles
     back to back, so tile boundaries inside one persistent CTA are checked."""
     S, seed = 2048, 700 + Hq + B
     p = api.LayerParams(Hq, Hkv, 128, W, 1e4, 128)
