@@ -20,6 +20,9 @@
 
 namespace swa {
 
+// calls with at most this many tokens run one block per token
+constexpr long long kRopeTokenBlocksMax = 4096;
+
 namespace rope_detail {
 
 constexpr int kChunks = kHeadDim / 8;  // 16-byte chunks per head row
@@ -290,6 +293,104 @@ __global__ void __launch_bounds__(256, 2) rope_keys_kernel(const RopeArgs a) {
   }
 }
 
+// One block per token (grid.y: ranges of its heads), for calls with few
+// tokens (decode steps, drafts): the block forms the token's cos/sin once
+// (shared memory), then every thread
+// takes one (head, 16-byte chunk) task per round of 16 heads -- q heads in
+// place, then k heads (and the cache append with its value) -- with all loads
+// of up to kTokRounds rounds issued before one barrier and all stores after
+// it, so rotating in place never reads a chunk another thread already wrote
+// (the next batch takes other heads).
+// Same arithmetic and slot rules as rope_kernel, so the results are bit for
+// bit those of the other paths.  Needs whole partner chunks (rotary_dim / 2 a
+// multiple of 8) and writes no cos/sin table.
+constexpr int kTokThreads = 256;
+constexpr int kTokRounds = 8;  // 8 rounds x 16 heads per load batch
+
+__global__ void __launch_bounds__(kTokThreads) rope_tokens_kernel(const RopeArgs a) {
+  __shared__ float2 cs[kMaxRotaryHalf];
+  const long long tk = blockIdx.x;
+  const int b = (int)(tk / a.S);
+  const int s_idx = (int)(tk % a.S);
+  const int p = a.pos ? a.pos[tk] : a.pos0 + s_idx;
+  const int r = a.rotate ? a.rotary_dim : 0;
+  const int half = r / 2;
+  if ((int)threadIdx.x < half) {
+    float c, sn;
+    rope_cos_sin((double)p * a.inv_freq[threadIdx.x], &c, &sn);
+    cs[threadIdx.x] = make_float2(c, sn);
+  }
+  // cache slot of this token: p mod W on a ring, p on a linear cache
+  long long slot = 0;
+  bool cache_it = false;
+  if (a.k_cache) {
+    slot = a.window > 0 ? (long long)(p % a.window) : (long long)p;
+    const bool fits = p >= 0 && slot < a.cache_capacity;
+    if (!fits && threadIdx.x == 0) record_error(kErrRope + 1);
+    cache_it = fits && !(a.window > 0 && !a.pos && p <= a.pos0 + a.S - 1 - a.window);
+  }
+  const long long dst_tok = (long long)b * (a.dst_rows > 0 ? a.dst_rows : a.S) + a.dst_row_off + s_idx;
+  const int nq = (a.q && r > 0) ? a.Hq : 0;  // without rotation q is left as it is
+  const int nk = a.k_src ? a.Hkv : 0;
+  const int chunk = threadIdx.x & (kChunks - 1);
+  const int d0 = chunk * 8;
+  const int role = d0 < half ? 1 : (d0 < r ? 2 : 0);
+  const int k0 = role == 2 ? d0 - half : d0;
+  const int pchunk = role == 1 ? chunk + half / 8 : chunk - half / 8;
+  const float sgn = role == 1 ? -1.f : 1.f;
+  __syncthreads();
+  // grid.y splits the token's heads into ranges of whole 16-head rounds
+  const int rounds = (nq + nk + kTokThreads / kChunks - 1) / (kTokThreads / kChunks);
+  const int per = (rounds + gridDim.y - 1) / gridDim.y;
+  const int lo = (int)blockIdx.y * per * (kTokThreads / kChunks);
+  const int hi = min(nq + nk, lo + per * (kTokThreads / kChunks));
+  for (int base = lo; base < hi; base += kTokRounds * (kTokThreads / kChunks)) {
+    uint4 own[kTokRounds], par[kTokRounds], val[kTokRounds];
+#pragma unroll
+    for (int u = 0; u < kTokRounds; ++u) {
+      const int hh = base + u * (kTokThreads / kChunks) + (int)(threadIdx.x / kChunks);  // q heads, then k heads
+      own[u] = par[u] = val[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (hh < hi) {
+        const uint16_t* row = hh < nq ? a.q + (tk * a.Hq + hh) * kHeadDim : a.k_src + (tk * a.Hkv + (hh - nq)) * kHeadDim;
+        own[u] = *reinterpret_cast<const uint4*>(row + chunk * 8);
+        if (role != 0) par[u] = *reinterpret_cast<const uint4*>(row + pchunk * 8);
+        if (hh >= nq && cache_it)
+          val[u] = __ldg(reinterpret_cast<const uint4*>(a.v + (tk * a.Hkv + (hh - nq)) * kHeadDim) + chunk);
+      }
+    }
+    __syncthreads();  // every chunk of these heads is read before any is written
+#pragma unroll
+    for (int u = 0; u < kTokRounds; ++u) {
+      const int hh = base + u * (kTokThreads / kChunks) + (int)(threadIdx.x / kChunks);
+      if (hh >= hi) continue;
+      uint4 yk = own[u];
+      if (r > 0 && role != 0) {
+        float x[8], xp[8], y[8];
+        unpack8(own[u], x);
+        unpack8(par[u], xp);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float2 t = cs[k0 + e];
+          y[e] = fmaf(x[e], t.x, sgn * (xp[e] * t.y));
+        }
+        yk = pack8(y);
+      }
+      if (hh < nq) {
+        *reinterpret_cast<uint4*>(a.q + (tk * a.Hq + hh) * kHeadDim + chunk * 8) = yk;
+      } else {
+        const int h = hh - nq;
+        *reinterpret_cast<uint4*>(a.k_dst + (dst_tok * a.Hkv + h) * kHeadDim + chunk * 8) = yk;
+        if (cache_it) {
+          *reinterpret_cast<uint4*>(a.k_cache + (((long long)b * a.Hkv + h) * a.cache_capacity + slot) * kHeadDim +
+                                    chunk * 8) = yk;
+          *reinterpret_cast<uint4*>(a.v_cache + (((long long)b * a.Hkv + h) * a.cache_capacity + slot) * kHeadDim +
+                                    chunk * 8) = val[u];
+        }
+      }
+    }
+  }
+}
+
 }  // namespace rope_detail
 
 cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
@@ -305,6 +406,16 @@ cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
   if (hsplit > max_heads) hsplit = max_heads;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   const int r = a.rotate ? a.rotary_dim : 0;
+  if (!a.table && n_tok <= kRopeTokenBlocksMax && ((r / 2) % 8) == 0) {
+    // few tokens: spread each token's heads over up to 4 blocks so that about
+    // two blocks per SM run
+    const int heads = (a.q && r > 0 ? a.Hq : 0) + (a.k_src ? a.Hkv : 0);
+    const int rounds = (heads + 15) / 16;
+    int ks = 1;
+    while (ks < 4 && ks * 2 <= rounds && n_tok * ks < 296) ks *= 2;
+    rope_detail::rope_tokens_kernel<<<dim3((unsigned)n_tok, (unsigned)ks), rope_detail::kTokThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
   const bool keys_only = !a.q && a.k_src && a.k_dst != a.k_src && ((r / 2) % 8) == 0;
   if (keys_only) {
     // one head split while a lane's heads fit one load group: each split
