@@ -349,6 +349,37 @@ def bench_prefill_e2e(c, steps: int, dev):
     return ev0.elapsed_time(ev1), h2d, d2h
 
 
+def time_calls(run, steps: int, warmup: int, stream):
+    """Device time per call of `run(i)`, i = 0 .. steps - 1: launched eagerly,
+    and replayed from a CUDA graph of the same `steps` calls (how a serving
+    loop issues decode steps: no per-call host work between the kernels).
+    Returns (ms_graph, ms_eager)."""
+    for i in range(max(warmup, 3)):
+        run(i)
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(steps):
+        run(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    eager = ev0.elapsed_time(ev1) / steps
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            run(i)
+    g.replay()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    g.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    graph = ev0.elapsed_time(ev1) / steps
+    del g
+    return graph, eager
+
+
 def bench_decode(c, steps: int, warmup: int, dev):
     from full_gqa_attention_swa_b200 import api
 
@@ -366,24 +397,13 @@ def bench_decode(c, steps: int, warmup: int, dev):
 
     def step(i):
         d = sets[i % n_sets]
-        api.attn_decode(p, d["q"], d["gate"], d["k_cache"], d["v_cache"], lens_d, max_len, out=out, workspace=ws,
-                        stream=stream)
+        api.attn_decode(p, d["q"], d["gate"], d["k_cache"], d["v_cache"], lens_d, max_len, out=out, workspace=ws)
 
-    for i in range(warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for i in range(steps):
-        step(i)
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = ev0.elapsed_time(ev1) / steps
+    ms, ms_eager = time_calls(step, steps, warmup, stream)
     nbytes = decode_bytes(c, lens.tolist())
     del sets
     torch.cuda.empty_cache()
-    return ms, nbytes
+    return ms, nbytes, ms_eager
 
 
 def bench_decode_mq(c, steps: int, warmup: int, dev):
@@ -406,23 +426,13 @@ def bench_decode_mq(c, steps: int, warmup: int, dev):
     def step(i):
         d, new = sets[i % n_sets]
         api.attn_decode_mq(p, new["q"], new["gate"], new["k"], new["v"], d["k_cache"], d["v_cache"], lens_d,
-                           max_len, out=out, workspace=ws, stream=stream)
+                           max_len, out=out, workspace=ws)
 
-    for i in range(warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for i in range(steps):
-        step(i)
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = ev0.elapsed_time(ev1) / steps
+    ms, ms_eager = time_calls(step, steps, warmup, stream)
     nbytes = decode_mq_bytes(c, lens.tolist())
     del sets
     torch.cuda.empty_cache()
-    return ms, nbytes
+    return ms, nbytes, ms_eager
 
 
 # --------------------------------------------------------------- CPU oracle
@@ -543,7 +553,7 @@ def main():
         if dist is not None:
             dist.barrier()
         run = bench_decode_mq if mq else bench_decode
-        d_ms, nbytes = run(dc, max(args.steps, 1), max(args.warmup, 3), dev)
+        d_ms, nbytes, _ = run(dc, max(args.steps, 1), max(args.warmup, 3), dev)
         d_ms = max_over_ranks(d_ms, dist, dev)
         gbs = nbytes * world / (d_ms / 1e3) / 1e9
         if rank == 0:
@@ -598,10 +608,11 @@ def main():
             for kind, dc in (("decode", configs.DECODE_SLIDING), ("mq", configs.MQ_SLIDING),
                              ("decode", configs.DECODE_FULL), ("mq", configs.MQ_FULL)):
                 steps = 200 if dc.window > 0 else 10
-                d_ms, nbytes = (bench_decode if kind == "decode" else bench_decode_mq)(dc, steps, 3, dev)
+                d_ms, nbytes, e_ms = (bench_decode if kind == "decode" else bench_decode_mq)(dc, steps, 3, dev)
                 gbs = nbytes / (d_ms / 1e3) / 1e9
                 (extra if kind == "decode" else mqs)[dc.name] = {
-                    "ms": d_ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                    "ms": d_ms, "ms_eager": e_ms, "timing": "CUDA graph replay of the steps (ms_eager: launched one by one)",
+                    "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                     "peak_source": f"{peak_src} hbm copy"}
             line["decode"] = extra
             line["decode_mq"] = mqs

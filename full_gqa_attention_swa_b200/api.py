@@ -173,6 +173,29 @@ def _device(*tensors, stream=None):
     return dev
 
 
+class _Current:
+    """Context that makes a CUDA device current only when it is not already
+    (the common case costs one device query, not a device switch)."""
+
+    __slots__ = ("dev", "prev")
+
+    def __init__(self, dev):
+        self.dev = dev
+        self.prev = None
+
+    def __enter__(self):
+        cur = torch.cuda.current_device()
+        if cur != self.dev.index:
+            self.prev = cur
+            torch.cuda.set_device(self.dev)
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            torch.cuda.set_device(self.prev)
+        return False
+
+
 def version() -> str:
     return load().swa_version().decode()
 
@@ -200,7 +223,7 @@ def rope_qk(layer: LayerParams, q=None, k=None, pos=None, pos0: int = 0, v=None,
         C = k_cache.shape[2]
         _need(k_cache, "k_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
         _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
-    with torch.cuda.device(_device(q, k, pos, v, k_cache, v_cache, stream=stream)):
+    with _Current(_device(q, k, pos, v, k_cache, v_cache, stream=stream)):
         _check(load().swa_rope_qk(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(pos), int(pos0), _ptr(v),
                                   _ptr(k_cache), _ptr(v_cache), C, _stream(stream)))
 
@@ -225,7 +248,7 @@ def attn_prefill(layer: LayerParams, q, k, v, gate=None, out=None, workspace=Non
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with torch.cuda.device(_device(q, k, v, gate, out, workspace, stream=stream)):
+    with _Current(_device(q, k, v, gate, out, workspace, stream=stream)):
         _check(load().swa_attn_prefill(ctypes.byref(layer.c()), B, S, _ptr(q), _ptr(k), _ptr(v), _ptr(gate),
                                        _ptr(out), _ptr(workspace), nbytes, _stream(stream)))
     return out
@@ -257,7 +280,7 @@ def attn_prefill_chunk(layer: LayerParams, pos0: int, q, k, v, gate, k_cache, v_
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with torch.cuda.device(_device(q, k, v, gate, k_cache, v_cache, out, workspace, stream=stream)):
+    with _Current(_device(q, k, v, gate, k_cache, v_cache, out, workspace, stream=stream)):
         _check(load().swa_attn_prefill_chunk(ctypes.byref(layer.c()), B, S, int(pos0), _ptr(q), _ptr(k), _ptr(v),
                                              _ptr(gate), _ptr(k_cache), _ptr(v_cache), C, _ptr(out), _ptr(workspace),
                                              nbytes, _stream(stream)))
@@ -288,7 +311,7 @@ def attn_decode(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens, max_len
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with torch.cuda.device(_device(q, gate, k_cache, v_cache, seq_lens, out, workspace, stream=stream)):
+    with _Current(_device(q, gate, k_cache, v_cache, seq_lens, out, workspace, stream=stream)):
         _check(load().swa_attn_decode(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache), _ptr(v_cache), C,
                                       _ptr(seq_lens), int(max_len), _ptr(out), _ptr(workspace), nbytes,
                                       _stream(stream)))
@@ -322,7 +345,7 @@ def attn_decode_mq(layer: LayerParams, q, gate, k_new, v_new, k_cache, v_cache, 
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with torch.cuda.device(_device(q, gate, k_new, v_new, k_cache, v_cache, seq_lens, out, workspace, stream=stream)):
+    with _Current(_device(q, gate, k_new, v_new, k_cache, v_cache, seq_lens, out, workspace, stream=stream)):
         _check(load().swa_attn_decode_mq(ctypes.byref(layer.c()), B, T, _ptr(q), _ptr(gate), _ptr(k_new), _ptr(v_new),
                                          _ptr(k_cache), _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
                                          _ptr(workspace), nbytes, _stream(stream)))
@@ -345,7 +368,7 @@ def attn_decode_no_alloc(layer: LayerParams, q, gate, k_cache, v_cache, seq_lens
     _need(v_cache, "v_cache", torch.bfloat16, (B, layer.num_kv_heads, C, D))
     _need(seq_lens, "seq_lens", torch.int32, (B,))
     _need(out, "out", torch.bfloat16, (B, layer.num_q_heads, D))
-    with torch.cuda.device(_device(q, gate, k_cache, v_cache, seq_lens, out, stream=stream)):
+    with _Current(_device(q, gate, k_cache, v_cache, seq_lens, out, stream=stream)):
         _check(load().swa_attn_decode_no_alloc(ctypes.byref(layer.c()), B, _ptr(q), _ptr(gate), _ptr(k_cache),
                                                _ptr(v_cache), C, _ptr(seq_lens), int(max_len), _ptr(out),
                                                _stream(stream)))
