@@ -98,7 +98,7 @@ PREFILL_TRAFFIC = {
     "workload": "step37_sliding_B1_S8192_Hq96_Hkv8_W512",
     "bytes": 402.3e6,
     # prefill.cuh and ptx.cuh (the kernel and its PTX helpers) as captured; any change makes the figure stale
-    "source_sha256": "d4566b0dd4deca3c3ea5079d21dad10e4756b31362501c4283f8a5613b40fb4d",
+    "source_sha256": "b6e81c15e05064bb2c486928bca3282e76ed40f6d0476859f1bc00d065199b28",
 }
 PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh")
 

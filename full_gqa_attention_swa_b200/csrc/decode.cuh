@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_split_kernel(cons
   DecodeSmem<NS>& sm =
       *reinterpret_cast<DecodeSmem<NS>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int L = a.seq_lens[b];
   const int n_vis = (a.window > 0 && L > a.window) ? a.window : L;
@@ -319,6 +321,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_split_kernel(cons
 
 // grid (Hq, B), 128 threads: merge the splits of one (sequence, q-head).
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a) {
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int L = a.seq_lens[b];
   const int n_vis = (a.window > 0 && L > a.window) ? a.window : L;
@@ -352,11 +356,9 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& k_map, const C
   });
   if (e != cudaSuccess) return e;
   dim3 grid(a.max_splits, a.Hkv, a.B);
-  decode_split_kernel<kStages><<<grid, kThreads, smem, stream>>>(a, k_map, v_map);
-  e = cudaGetLastError();
+  e = launch_kernel(true, decode_split_kernel<kStages>, grid, dim3(kThreads), smem, stream, a, k_map, v_map);
   if (e != cudaSuccess || a.max_splits == 1) return e;
-  decode_combine_kernel<<<dim3(a.Hq, a.B), kHeadDim, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(true, decode_combine_kernel, dim3(a.Hq, a.B), dim3(kHeadDim), 0, stream, a);
 }
 
 }  // namespace swa

@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(MT * 32, ctas_per_sm(MT))
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   MqSmem& sm = *reinterpret_cast<MqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int T = a.T;
   const int L0 = a.seq_lens[b] - T;  // cached tokens before the new ones
@@ -363,6 +365,8 @@ __global__ void __launch_bounds__(MT * 32, ctas_per_sm(MT))
 // grid (Hq, T, B), 128 threads: merge the splits of one (sequence, query, q-head).
 // A split whose keys all lie outside a query's band left (-inf, 0) and weighs 0.
 __global__ void __launch_bounds__(128) decode_mq_combine_kernel(const DecodeMqArgs a) {
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int h = blockIdx.x, t = blockIdx.y, b = blockIdx.z, d = threadIdx.x;
   const int L0 = a.seq_lens[b] - a.T;
   if (L0 < 0 || (a.window < 0 && L0 > a.capacity)) return;
@@ -392,11 +396,10 @@ cudaError_t launch_mq(const DecodeMqArgs& a, const CUtensorMap& k_map, const CUt
     return cudaFuncSetAttribute(decode_mq_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   });
   if (e != cudaSuccess) return e;
-  decode_mq_kernel<MT><<<dim3(a.max_splits, a.Hkv, a.B), MT * 32, smem, stream>>>(a, k_map, v_map);
-  e = cudaGetLastError();
+  e = launch_kernel(true, decode_mq_kernel<MT>, dim3(a.max_splits, a.Hkv, a.B), dim3(MT * 32), smem, stream, a, k_map,
+                       v_map);
   if (e != cudaSuccess || a.max_splits == 1) return e;
-  decode_mq_combine_kernel<<<dim3(a.Hq, a.T, a.B), kHeadDim, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(true, decode_mq_combine_kernel, dim3(a.Hq, a.T, a.B), dim3(kHeadDim), 0, stream, a);
 }
 
 }  // namespace decode_mq_detail

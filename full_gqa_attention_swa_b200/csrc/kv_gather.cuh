@@ -46,8 +46,7 @@ cudaError_t launch_kv_gather(const KvGatherArgs& a, cudaStream_t stream) {
   if (lanes == 0) return cudaSuccess;
   const long long blocks = (lanes + 255) / 256;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  kv_gather_detail::kv_gather_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(false, kv_gather_detail::kv_gather_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, a);
 }
 
 }  // namespace swa

@@ -795,8 +795,8 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& q_map, con
   }, &n_sm);
   if (e != cudaSuccess) return e;
   const int grid = (int)(n_tiles < n_sm ? n_tiles : n_sm);
-  prefill_kernel<kMode><<<grid, kThreads, smem, stream>>>(a, q_map, k_map, v_map, o_map);
-  return cudaGetLastError();
+  return launch_kernel(false, prefill_kernel<kMode>, dim3(grid), dim3(kThreads), smem, stream, a, q_map, k_map, v_map,
+                          o_map);
 }
 
 }  // namespace prefill_detail

@@ -360,6 +360,18 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t y) {
                  __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may be scheduled while the kernel before it on the stream is
+// still running; grid_dependency_wait() returns once that kernel has
+// completed and its memory writes are visible (at once without the launch
+// attribute), and allow_dependent_launch() lets the next such kernel be
+// scheduled as soon as every block of this one has started.  The kernels
+// launched that way (the decode path) call both first, before they read
+// global memory; the others are launched plainly and wait for the previous
+// kernel as usual.
+__device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

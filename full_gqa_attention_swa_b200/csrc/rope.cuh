@@ -308,6 +308,8 @@ constexpr int kTokThreads = 256;
 constexpr int kTokRounds = 8;  // 8 rounds x 16 heads per load batch
 
 __global__ void __launch_bounds__(kTokThreads) rope_tokens_kernel(const RopeArgs a) {
+  allow_dependent_launch();
+  grid_dependency_wait();
   __shared__ float2 cs[kMaxRotaryHalf];
   const long long tk = blockIdx.x;
   const int b = (int)(tk / a.S);
@@ -413,19 +415,18 @@ cudaError_t launch_rope(const RopeArgs& a, cudaStream_t stream) {
     const int rounds = (heads + 15) / 16;
     int ks = 1;
     while (ks < 4 && ks * 2 <= rounds && n_tok * ks < 296) ks *= 2;
-    rope_detail::rope_tokens_kernel<<<dim3((unsigned)n_tok, (unsigned)ks), rope_detail::kTokThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(true, rope_detail::rope_tokens_kernel, dim3((unsigned)n_tok, (unsigned)ks),
+                            dim3(rope_detail::kTokThreads), 0, stream, a);
   }
   const bool keys_only = !a.q && a.k_src && a.k_dst != a.k_src && ((r / 2) % 8) == 0;
   if (keys_only) {
     // one head split while a lane's heads fit one load group: each split
     // recomputes the lane's cos/sin
     const unsigned ks = (unsigned)(a.Hkv <= rope_detail::kKeyGroup ? 1 : hsplit);
-    rope_detail::rope_keys_kernel<<<dim3((unsigned)blocks, ks), threads, 0, stream>>>(a);
+    return launch_kernel(false, rope_detail::rope_keys_kernel, dim3((unsigned)blocks, ks), dim3(threads), 0, stream, a);
   }
-  else
-    rope_detail::rope_kernel<<<dim3((unsigned)blocks, (unsigned)hsplit), threads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(false, rope_detail::rope_kernel, dim3((unsigned)blocks, (unsigned)hsplit), dim3(threads), 0,
+                          stream, a);
 }
 
 }  // namespace swa
