@@ -175,3 +175,24 @@ def test_q_and_out_beyond_2_31_elements(cuda_device):
                          rows=rows)
     assert_close(got, ref, "q/out beyond 2^31 elements")
     check_no_device_error()
+
+
+@pytest.mark.parametrize("S", [5, 37])
+def test_many_short_sequences(cuda_device, S):
+    """B = 300 sequences of a few tokens: one ragged 128-row tile per
+    (sequence, head pair); the loads read zeros past S and the stores clip
+    there, so neighbouring sequences are left intact."""
+    B, Hq, Hkv = 300, 8, 2
+    for W in (3, -1):
+        p = api.LayerParams(Hq, Hkv, 128, W, 1e4, 128)
+        d = inputs.prefill_inputs(B, S, Hq, Hkv, 128, seed=800 + S)
+        dev = {k: t.to(cuda_device) for k, t in d.items()}
+        out = api.attn_prefill(p, dev["q"], dev["k"], dev["v"], dev["gate"])
+        torch.cuda.synchronize()
+        rng = np.random.default_rng(S)
+        rows = np.stack([rng.integers(0, B, 200), rng.integers(0, S, 200), rng.integers(0, Hq, 200)], 1)
+        rows = np.concatenate([rows, np.array([(0, 0, 0), (B - 1, S - 1, Hq - 1)], np.int64)]).astype(np.int64)
+        ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy(), rows=rows)
+        got = out.cpu()[torch.from_numpy(rows[:, 0]), torch.from_numpy(rows[:, 1]), torch.from_numpy(rows[:, 2])]
+        assert_close(got, ref, f"B{B} S{S} W{W}")
+    check_no_device_error()
