@@ -462,6 +462,30 @@ def oracle_sample_rate(c, budget_s: float, threads: int = 0):
     return flops / dt / 1e12, n, dt, (threads or oracle.num_threads())
 
 
+def oracle_parity_sample(c, dev, n_rows: int = 512) -> dict:
+    """Part of the CPU-baseline leg: the timed workload's first input set once
+    more through swa_attn_prefill, and the oracle on a seeded sample of its
+    rows; returns the worst |gpu - oracle| and how many elements exceed the
+    parity tolerance."""
+    import oracle
+    from full_gqa_attention_swa_b200 import api
+
+    p = _layer(c)
+    d = inputs.prefill_inputs(c.B, c.S, c.Hq, c.Hkv, 128, c.seed, device=dev)   # set 0 of the timed loop
+    out = api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"])
+    torch.cuda.synchronize(dev)
+    rng = np.random.default_rng(c.seed + 1)
+    rows = np.stack([rng.integers(0, c.B, n_rows), rng.integers(0, c.S, n_rows), rng.integers(0, c.Hq, n_rows)], 1)
+    lay = oracle.Layer(c.Hq, c.Hkv, 128, c.window, c.theta, c.rotary_dim)
+    ref = oracle.prefill(lay, inputs.as_bits(d["q"].cpu()), inputs.as_bits(d["k"].cpu()), inputs.as_bits(d["v"].cpu()),
+                         d["gate"].cpu().numpy(), rows=rows)
+    idx = [torch.from_numpy(rows[:, i]).to(dev) for i in range(3)]
+    got = out[idx[0], idx[1], idx[2]].float().cpu().double().numpy()
+    err = np.abs(got - ref)
+    return {"rows": n_rows, "max_abs_err": float(err.max()),
+            "out_of_tolerance": int((err > 1e-2 + 1e-2 * np.abs(ref)).sum()), "tolerance": "1e-2 + 1e-2 |oracle|"}
+
+
 # --------------------------------------------------------------------- main
 
 def main():
@@ -620,7 +644,8 @@ def main():
         if world == 1 and args.cpu_budget > 0:
             r, n, dt, thr = oracle_sample_rate(c, args.cpu_budget)
             line["cpu_baseline"] = {"value": r, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-                                    "sample": f"{n} seeded random (b, i, h) rows of {c.name}, {dt:.1f} s"}
+                                    "sample": f"{n} seeded random (b, i, h) rows of {c.name}, {dt:.1f} s",
+                                    "parity_sample": oracle_parity_sample(c, dev)}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
