@@ -169,38 +169,54 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// Rotate query row `row` (position i) of a Q tile in shared memory (two
+// Rotate query row `row` (position i) of the Q tiles in shared memory (two
 // 64-dim boxes, 128-byte swizzle): pairs (k, k + r/2) for k < r/2.  Vector
-// form for 16 | r: tb holds the row's 16-byte table slices (two pairs each),
-// loaded before the tile's arrival is awaited; the warp's 32 rows load each
-// slice index from 512 contiguous bytes.
-__device__ __forceinline__ void rope_table_load(float4 (&tb)[32], const float4* __restrict__ tgroup, int half) {
+// form for 16 | r.  Both head slots' tiles hold the same query rows, so the
+// slots split a row's 8-pair chunks between them (slot s takes chunks
+// c0 = s, s+2, s+4, s+6) and each rotates its chunks in both tiles: every
+// table slice crosses from L2 once per work tile.  tb holds the thread's
+// 16-byte slices (two pairs each), loaded before the tiles' arrival is
+// awaited; the warp's 32 rows load each slice index from 512 contiguous
+// bytes.
+__device__ __forceinline__ void rope_table_load(float4 (&tb)[16], const float4* __restrict__ tgroup, int half,
+                                                int slot) {
   // slices past half/2 repeat the last one: unconditional loads stay in registers
   const int last = half / 2 - 1;
 #pragma unroll
-  for (int k = 0; k < 32; ++k) tb[k] = __ldg(tgroup + (size_t)min(k, last) * 32);
+  for (int ci = 0; ci < 4; ++ci)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) tb[4 * ci + w] = __ldg(tgroup + (size_t)min((2 * ci + slot) * 4 + w, last) * 32);
 }
 
-__device__ __forceinline__ void rotate_q_row_vec(uint8_t* tile, int row, int half, const float4 (&tb)[32]) {
+// Rotates dims 8 c0 .. 8 c0 + 7 with their partners 8 c0 + half .. of one row;
+// t4[w] holds (cos, sin) of pairs 8 c0 + 2w and 8 c0 + 2w + 1.
+__device__ __forceinline__ void rotate_q_chunk(uint8_t* tile, int row, int c0, int half, const float4* t4) {
+  const int ea = c0 * 8, eb = ea + half;
+  uint4* pa = reinterpret_cast<uint4*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3));
+  uint4* pb = reinterpret_cast<uint4*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3));
+  uint4 A = *pa, Bv = *pb;
+  uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
+  uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
 #pragma unroll
-  for (int c0 = 0; c0 < 8; ++c0) {
+  for (int w = 0; w < 4; ++w) {
+    const float4 t = t4[w];
+    const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
+    const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
+    a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
+    b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
+  }
+  *pa = A;
+  *pb = Bv;
+}
+
+__device__ __forceinline__ void rotate_q_rows_vec(uint8_t* q0, uint8_t* q1, int row, int half, int slot,
+                                                  const float4 (&tb)[16]) {
+#pragma unroll
+  for (int ci = 0; ci < 4; ++ci) {
+    const int c0 = 2 * ci + slot;
     if (c0 * 8 < half) {
-      const int ea = c0 * 8, eb = ea + half;
-      uint4* pa = reinterpret_cast<uint4*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3));
-      uint4* pb = reinterpret_cast<uint4*>(tile + (eb >> 6) * kBoxBytes + sw128_off(row, (eb & 63) >> 3));
-      uint4 A = *pa, Bv = *pb;
-      uint32_t* a32 = reinterpret_cast<uint32_t*>(&A);
-      uint32_t* b32 = reinterpret_cast<uint32_t*>(&Bv);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float4 t = tb[c0 * 4 + w];  // (cos, sin) of pairs ea+2w and ea+2w+1
-        const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
-        const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
-        a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
-        b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
-      }
-      *pa = A;
-      *pb = Bv;
+      rotate_q_chunk(q0, row, c0, half, tb + 4 * ci);
+      rotate_q_chunk(q1, row, c0, half, tb + 4 * ci);
     }
   }
 }
@@ -284,7 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Per work tile: K(0), then [K(j+1), V(j)] per key tile (K runs one
       // ahead, its 2-deep ring frees early; V's single buffer frees when both
       // slots' P.V of the previous key tile complete).  The next tile's Q is
-      // loaded as soon as this tile's last QK^T has read Q.
+      // loaded as soon as this tile's last QK^T has read Q.  No L2 prefetches
+      // (of the next V, or of a later tile's Q and cos/sin rows): with them
+      // the loads queued behind land later and the step is about 2 % slower.
       prefetch_tensormap(&q_map);
       prefetch_tensormap(&k_map);
       prefetch_tensormap(&v_map);
@@ -301,21 +319,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(sm.q[s], &q_map, &sm.q_full[s], 0, h, N.r0, N.b);
           tma_load_4d(sm.q[s] + kBoxBytes, &q_map, &sm.q_full[s], 64, h, N.r0, N.b);
           q_last[s] = it_q;
-        }
-        // warm L2 for the Q tiles and cos/sin rows of the tile after it
-        if (t_q + (int)gridDim.x < n_tiles) {
-          const Tile M = decode_tile<kMode>(a, t_q + gridDim.x);
-          for (int s = 0; s < 2; ++s) {
-            const int h = s ? M.h1 : M.h0;
-            tma_prefetch_4d(&q_map, 0, h, M.r0, M.b);
-            tma_prefetch_4d(&q_map, 64, h, M.r0, M.b);
-          }
-          if (a.rotary_dim > 0) {
-            // the tile's rows are whole groups of 32 (r0 % 128 == 0)
-            const int half = a.rotary_dim / 2;
-            const uint32_t bytes = (uint32_t)(((min(BM, a.S - M.r0) + 31) >> 5) * rope_table_couples(half) * 512);
-            bulk_prefetch_l2(a.table + rope_table_index(M.r0, 0, half), bytes);
-          }
         }
         return true;
       };
@@ -337,15 +340,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(dst, map, full, 0, T.kvh, key0, T.b);
           tma_load_4d(dst + kBoxBytes, map, full, 64, T.kvh, key0, T.b);
         }
-        if (is_v) {
+        if (is_v)
           v_end = idx + 1;
-          if (kMode != kChunkCache && j + 1 < T.n_kv) {  // the next V comes through L2
-            tma_prefetch_4d(&v_map, 0, T.kvh, key0 + BN, T.b);
-            tma_prefetch_4d(&v_map, 64, T.kvh, key0 + BN, T.b);
-          }
-        } else {
+        else
           k_end = idx + 1;
-        }
         return true;
       };
       if (blockIdx.x < (unsigned)n_tiles && !load_q(blockIdx.x, 0)) ok = false;
@@ -522,28 +520,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile T = decode_tile<kMode>(a, t);
       const int r = T.r0 + row;  // query row
       const int i = T.i0 + row;  // its key-space position
-      // ---- RoPE of this slot's Q tile (rows at or beyond S stay as loaded:
-      // zero); the first table slices are requested before Q is awaited
+      // ---- RoPE of the Q tiles (rows at or beyond S stay as loaded: zero);
+      // the table slices are requested before Q is awaited.  Vector form:
+      // this slot's half of each row's chunks in both tiles; scalar form:
+      // this slot's own tile.
       {
         const int half = a.rotary_dim / 2;
         const bool rot = a.rotary_dim > 0 && r < a.S;
         const bool vec = (half & 7) == 0;
         const float4* tgroup = reinterpret_cast<const float4*>(a.table) +
                                ((((size_t)(r >> 5) * rope_table_couples(half)) << 5) + (r & 31));
-        float4 tb[32];
+        float4 tb[16];
         if (rot && vec) {
-          rope_table_load(tb, tgroup, half);
+          rope_table_load(tb, tgroup, half, s);
         } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) tb[k] = make_float4(1.f, 0.f, 1.f, 0.f);
+          for (int k = 0; k < 16; ++k) tb[k] = make_float4(1.f, 0.f, 1.f, 0.f);
         }
-        if (!warp_wait(&sm.q_full[s], it & 1, abort_flag)) {
+        if (!warp_wait(&sm.q_full[0], it & 1, abort_flag) || !warp_wait(&sm.q_full[1], it & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 6);
+          ok = false;
           break;
         }
         if (rot) {
           if (vec)
-            rotate_q_row_vec(sm.q[s], row, half, tb);
+            rotate_q_rows_vec(sm.q[0], sm.q[1], row, half, s, tb);
           else
             rotate_q_row_scalar(sm.q[s], row, r, half, a.table);
         }
