@@ -465,8 +465,8 @@ def oracle_sample_rate(c, budget_s: float, threads: int = 0):
 def oracle_parity_sample(c, dev, n_rows: int = 512) -> dict:
     """Part of the CPU-baseline leg: the timed workload's first input set once
     more through swa_attn_prefill, and the oracle on a seeded sample of its
-    rows; returns the worst |gpu - oracle| and how many elements exceed the
-    parity tolerance."""
+    rows; returns the worst and the RMS |gpu - oracle| and how many elements
+    exceed the parity tolerance."""
     import oracle
     from full_gqa_attention_swa_b200 import api
 
@@ -482,7 +482,7 @@ def oracle_parity_sample(c, dev, n_rows: int = 512) -> dict:
     idx = [torch.from_numpy(rows[:, i]).to(dev) for i in range(3)]
     got = out[idx[0], idx[1], idx[2]].float().cpu().double().numpy()
     err = np.abs(got - ref)
-    return {"rows": n_rows, "max_abs_err": float(err.max()),
+    return {"rows": n_rows, "max_abs_err": float(err.max()), "rms_err": float(np.sqrt((err ** 2).mean())),
             "out_of_tolerance": int((err > 1e-2 + 1e-2 * np.abs(ref)).sum()), "tolerance": "1e-2 + 1e-2 |oracle|"}
 
 

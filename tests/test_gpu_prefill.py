@@ -52,8 +52,12 @@ def test_ragged_lengths(cuda_device, S, W):
 
 
 @pytest.mark.parametrize("theta,r", [(5e6, 64), (0.0, 128), (5e5, 32), (1e4, 16), (1e4, 24), (1e4, 6), (1e4, 2),
-                                     (1e4, 0)])
+                                     (1e4, 0), (1e4, 48), (1e4, 80), (5e5, 112)])
 def test_rope_variants(cuda_device, theta, r):
+    """Partial rotary widths through the in-kernel Q rotation: the vector form
+    splits a row's 8-pair chunks between the two head slots (48, 80 and 112
+    give the slots unequal counts; 16 leaves slot 1 none), widths not a
+    multiple of 16 take the scalar form."""
     p = api.LayerParams(8, 2, 128, 200, theta, r)
     _check_all_rows(cuda_device, p, 1, 384, seed=300 + r)
     check_no_device_error()
