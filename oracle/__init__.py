@@ -96,52 +96,57 @@ class Layer:
 _lib = None
 
 
+def _configure(lib):
+    """Set the argument and result types of every oracle entry point on a
+    loaded library (the built liboracle.so, or a test's variant of it)."""
+    P = ctypes.POINTER
+    lib.oracle_rope.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                ctypes.c_void_p, ctypes.c_double, ctypes.c_int32, ctypes.c_void_p]
+    lib.oracle_rope.restype = ctypes.c_int
+    lib.oracle_rope_table.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
+    lib.oracle_rope_table.restype = ctypes.c_int
+    lib.oracle_rope_vec_table.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_double]
+    lib.oracle_rope_vec_table.restype = None
+    lib.oracle_prefill.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+    lib.oracle_prefill.restype = ctypes.c_int
+    lib.oracle_prefill_materialised.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    lib.oracle_prefill_materialised.restype = ctypes.c_int
+    lib.oracle_decode.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_int32]
+    lib.oracle_decode.restype = ctypes.c_int
+    lib.oracle_decode_f64.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                      ctypes.c_void_p, ctypes.c_void_p]
+    lib.oracle_decode_f64.restype = ctypes.c_int
+    lib.oracle_decode_mq.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+    lib.oracle_decode_mq.restype = ctypes.c_int
+    lib.oracle_kv_cache_bytes.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.c_int32, ctypes.c_int32]
+    lib.oracle_kv_cache_bytes.restype = ctypes.c_int64
+    lib.oracle_visible_count.argtypes = [ctypes.c_int64, ctypes.c_int32]
+    lib.oracle_visible_count.restype = ctypes.c_int64
+    lib.oracle_rope_vec.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
+                                    ctypes.c_double]
+    lib.oracle_rope_vec.restype = None
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P = ctypes.POINTER
-        lib.oracle_rope.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
-                                    ctypes.c_void_p, ctypes.c_double, ctypes.c_int32, ctypes.c_void_p]
-        lib.oracle_rope.restype = ctypes.c_int
-        lib.oracle_rope_table.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
-                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
-        lib.oracle_rope_table.restype = ctypes.c_int
-        lib.oracle_rope_vec_table.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_double]
-        lib.oracle_rope_vec_table.restype = None
-        lib.oracle_prefill.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
-                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
-        lib.oracle_prefill.restype = ctypes.c_int
-        lib.oracle_prefill_materialised.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32,
-                                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
-        lib.oracle_prefill_materialised.restype = ctypes.c_int
-        lib.oracle_decode.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
-                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
-                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
-                                      ctypes.c_void_p, ctypes.c_int32]
-        lib.oracle_decode.restype = ctypes.c_int
-        lib.oracle_decode_f64.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
-                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
-                                          ctypes.c_void_p, ctypes.c_void_p]
-        lib.oracle_decode_f64.restype = ctypes.c_int
-        lib.oracle_decode_mq.argtypes = [P(_Layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
-                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
-                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
-                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
-        lib.oracle_decode_mq.restype = ctypes.c_int
-        lib.oracle_kv_cache_bytes.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
-                                              ctypes.c_int32, ctypes.c_int32]
-        lib.oracle_kv_cache_bytes.restype = ctypes.c_int64
-        lib.oracle_visible_count.argtypes = [ctypes.c_int64, ctypes.c_int32]
-        lib.oracle_visible_count.restype = ctypes.c_int64
-        lib.oracle_rope_vec.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
-                                        ctypes.c_double]
-        lib.oracle_rope_vec.restype = None
-        lib.oracle_num_threads.argtypes = []
-        lib.oracle_num_threads.restype = ctypes.c_int
-        _lib = lib
+        _lib = _configure(ctypes.CDLL(build()))
     return _lib
 
 
