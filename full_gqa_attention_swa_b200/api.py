@@ -69,6 +69,10 @@ class LayerParams:
     inv_freq: tuple = None
 
     def c(self) -> _Params:
+        """The swa_layer_params struct, built once per (immutable) instance."""
+        prm = self.__dict__.get("_c")
+        if prm is not None:
+            return prm
         freq = None
         if self.inv_freq is not None:
             if len(self.inv_freq) != self.rotary_dim // 2:
@@ -78,6 +82,7 @@ class LayerParams:
                       self.rotary_dim, float(self.softmax_scale),
                       None if freq is None else ctypes.cast(freq, ctypes.POINTER(ctypes.c_double)))
         prm._freq = freq  # the table lives as long as the struct that points to it
+        object.__setattr__(self, "_c", prm)  # not a field: equality and hashing ignore it
         return prm
 
 
@@ -138,10 +143,18 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream):
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    """The cudaStream_t to launch on: the given stream, else the current
+    stream of the current device (read as a raw handle, without building a
+    torch.cuda.Stream object)."""
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    if _raw_stream is not None:
+        return ctypes.c_void_p(_raw_stream(torch.cuda.current_device()))
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
 def _need(t, name, dtype, shape=None):
