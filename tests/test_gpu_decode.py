@@ -12,10 +12,14 @@ from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer
 pytestmark = pytest.mark.gpu
 
 
-def _run(cuda_device, p, B, C, lens, seed, gate=True, poison=False, rows=None):
+def _run(cuda_device, p, B, C, lens, seed, gate=True, poison=False, rows=None, scale=1.0):
+    """scale multiplies q and the cached keys (scores grow with its square)."""
     d = inputs.decode_inputs(B, p.num_q_heads, p.num_kv_heads, 128, C, seed)
     lens_t = torch.tensor(lens, dtype=torch.int32)
     kc, vc = d["k_cache"].clone(), d["v_cache"].clone()
+    if scale != 1.0:
+        d["q"] = (d["q"].float() * scale).to(torch.bfloat16)
+        kc = (kc.float() * scale).to(torch.bfloat16)
     if poison:   # slots nobody may read hold NaN
         for b, L in enumerate(lens):
             n = min(L, p.window) if p.window > 0 else L
@@ -57,6 +61,14 @@ def test_split_k_paths(cuda_device):
     _run(cuda_device, p, len(lens), 20480, lens, seed=70)
     pw = api.LayerParams(24, 2, 128, 2048, 5e5, 128)
     _run(cuda_device, pw, 3, 2048, [5, 2048, 100000], seed=71)
+    check_no_device_error()
+
+
+def test_large_scores(cuda_device):
+    """q and keys times 3: a few keys dominate each row, and the split-K merge
+    weighs partials whose maxima lie far apart."""
+    _run(cuda_device, api.LayerParams(24, 2, 128, 64, 1e4, 128), 4, 64, [3, 64, 65, 700], seed=74, scale=3.0)
+    _run(cuda_device, api.LayerParams(16, 2, 128, -1, 5e6, 64), 3, 12000, [9, 4097, 12000], seed=75, scale=3.0)
     check_no_device_error()
 
 

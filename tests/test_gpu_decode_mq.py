@@ -15,12 +15,17 @@ from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer
 pytestmark = pytest.mark.gpu
 
 
-def _run(cuda_device, p, B, T, C, lens, seed, gate=True, poison=False):
+def _run(cuda_device, p, B, T, C, lens, seed, gate=True, poison=False, scale=1.0):
     """Random cache of capacity C holding lens[b] - T earlier tokens, random
-    (already rotated) new tokens; returns the GPU output and the oracle's."""
+    (already rotated) new tokens; returns the GPU output and the oracle's.
+    scale multiplies q and every key (scores grow with its square)."""
     d = inputs.decode_inputs(B, p.num_q_heads, p.num_kv_heads, 128, C, seed)
     new = inputs.prefill_inputs(B, T, p.num_q_heads, p.num_kv_heads, 128, seed + 1, with_gate=gate)
     kc, vc = d["k_cache"].clone(), d["v_cache"].clone()
+    if scale != 1.0:
+        new["q"] = (new["q"].float() * scale).to(torch.bfloat16)
+        new["k"] = (new["k"].float() * scale).to(torch.bfloat16)
+        kc = (kc.float() * scale).to(torch.bfloat16)
     if poison:   # slots outside every query's band hold NaN
         for b, L in enumerate(lens):
             L0 = L - T
@@ -77,6 +82,14 @@ def test_row_tiles(cuda_device, G, T):
         lens = [T, T + 40, T + 200] if W < 0 else [T + 1, T + 63, T + 64, T + 300]
         out, ref = _run(cuda_device, p, len(lens), T, C, lens, seed=2200 + G * T + max(W, 0))
         assert_close(out, ref, f"mq tiles G{G} T{T} W{W}")
+    check_no_device_error()
+
+
+def test_large_scores(cuda_device):
+    for p, C, lens, seed in ((api.LayerParams(24, 2, 128, 64, 1e4, 128), 64, [4, 40, 68, 900], 830),
+                             (api.LayerParams(16, 2, 128, -1, 5e6, 64), 9000, [4, 3000, 9000], 831)):
+        out, ref = _run(cuda_device, p, len(lens), 4, C, lens, seed, scale=3.0)
+        assert_close(out, ref, f"multi-query large scores W{p.window}")
     check_no_device_error()
 
 

@@ -1,6 +1,6 @@
 """swa_attn_prefill on the GPU against the oracle: the tiny case in full,
 window sweeps around tile edges, ragged lengths, partial / no RoPE, odd GQA
-groups, no gate, the uniform-score window-count probe at full size, and the
+groups, no gate, large and steadily growing scores (the lazy rescale), the uniform-score window-count probe at full size, and the
 full-size prefill workloads on seeded row samples."""
 import numpy as np
 import pytest
@@ -87,6 +87,52 @@ def test_no_gate_and_custom_scale(cuda_device):
 
 
 @pytest.mark.slow
+def _score_extreme_inputs(kind, B, S, Hq, Hkv, seed):
+    """Inputs whose scores stress the online softmax.  'large': q and k times
+    3, so scores have a standard deviation near 9 (natural units) and a few
+    keys dominate each row.  'growing': every query and key points along one
+    direction, keys lengthening linearly with position, so a row's running
+    max climbs about 6 (log2 units) per 128-key tile -- under the kernel's
+    rescale threshold of 8 for one tile, over it across two."""
+    d = inputs.prefill_inputs(B, S, Hq, Hkv, 128, seed)
+    if kind == "large":
+        d["q"] = (d["q"].float() * 3).to(torch.bfloat16)
+        d["k"] = (d["k"].float() * 3).to(torch.bfloat16)
+    else:
+        ramp = torch.arange(S, dtype=torch.float32).view(1, S, 1, 1) / S
+        d["q"] = (1.41 + 0.1 * d["q"].float()).to(torch.bfloat16)
+        d["k"] = (1.41 * ramp + 0.1 * d["k"].float()).to(torch.bfloat16)
+    return d
+
+
+@pytest.mark.parametrize("kind,W,theta", [("large", 300, 1e4), ("large", -1, 1e4), ("growing", 300, 0.0),
+                                          ("growing", -1, 0.0)])
+def test_score_extremes(cuda_device, kind, W, theta):
+    """The kernels round the rotated q and k to bf16 before their MMAs.  At
+    these score magnitudes that rounding alone moves the exact attention
+    output by up to about 6e-2 (the oracle fed rounded operands shows the same
+    shift), so with RoPE on, the reference is the oracle's rotation rounded to
+    bf16 and then attended without rotation; with theta = 0 both sides see
+    identical operands and the reference is the plain oracle."""
+    B, S, Hq, Hkv = 2, 700, 4, 2
+    p = api.LayerParams(Hq, Hkv, 128, W, theta, 128)
+    d = _score_extreme_inputs(kind, B, S, Hq, Hkv, seed=720 + (W > 0))
+    dev = {k: t.to(cuda_device) for k, t in d.items()}
+    out = api.attn_prefill(p, dev["q"], dev["k"], dev["v"], dev["gate"])
+    torch.cuda.synchronize()
+    q, k = bits(d["q"]), bits(d["k"])
+    lay = oracle_layer(p)
+    if theta > 0:
+        pos = np.arange(S, dtype=np.int64)
+        rot = lambda x: bits(torch.from_numpy(
+            np.stack([oracle.rope(x[b], pos, theta, 128) for b in range(B)])).to(torch.bfloat16))
+        q, k = rot(q), rot(k)
+        lay = oracle.Layer(Hq, Hkv, 128, W, 0.0, 128)
+    ref = oracle.prefill(lay, q, k, bits(d["v"]), d["gate"].numpy())
+    assert_close(out, ref, f"prefill {kind} W{W}")
+    check_no_device_error()
+
+
 @pytest.mark.parametrize("cfg", [configs.STEP_SLIDING, configs.MUSE_SLIDING], ids=lambda c: c.name)
 def test_uniform_score_probe_window_counts(cuda_device, cfg):
     """Q = 0 makes every score 0: each output row is sigmoid(g) times the mean
