@@ -133,6 +133,24 @@ def test_score_extremes(cuda_device, kind, W, theta):
     check_no_device_error()
 
 
+def test_saturated_gate_logits(cuda_device):
+    """Gate logits of +-60 and +-1e4 saturate the sigmoid: the output is the
+    ungated attention, about 1e-26 of it (sigmoid(-60)), or exactly zero
+    (sigmoid(-1e4) underflows), never NaN."""
+    B, S, Hq, Hkv = 1, 300, 8, 2
+    p = api.LayerParams(Hq, Hkv, 128, 100, 1e4, 128)
+    d = inputs.prefill_inputs(B, S, Hq, Hkv, 128, 760)
+    levels = torch.tensor([60.0, -60.0, 1e4, -1e4, 0.0, 3.0, -3.0, 60.0])
+    d["gate"] = levels.view(1, 1, Hq).expand(B, S, Hq).contiguous()
+    dev = {k: t.to(cuda_device) for k, t in d.items()}
+    out = api.attn_prefill(p, dev["q"], dev["k"], dev["v"], dev["gate"])
+    torch.cuda.synchronize()
+    ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy())
+    assert_close(out, ref, "prefill saturated gates")
+    assert bool((out[:, :, 3] == 0).all()) and bool((out[:, :, 1].float().abs() < 1e-20).all())
+    check_no_device_error()
+
+
 @pytest.mark.parametrize("cfg", [configs.STEP_SLIDING, configs.MUSE_SLIDING], ids=lambda c: c.name)
 def test_uniform_score_probe_window_counts(cuda_device, cfg):
     """Q = 0 makes every score 0: each output row is sigmoid(g) times the mean
