@@ -202,8 +202,10 @@ __device__ __forceinline__ void rotate_q_chunk(uint8_t* tile, int row, int c0, i
     const float4 t = t4[w];
     const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
     const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
-    a32[w] = pack_bf16x2(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
-    b32[w] = pack_bf16x2(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
+    // the partner's product rounded, then one fma: the RoPE kernels' form,
+    // so a rotated q equals swa_rope_qk's bit for bit
+    a32[w] = pack_bf16x2(fmaf(x0, t.x, -(y0 * t.y)), fmaf(x1, t.z, -(y1 * t.w)));
+    b32[w] = pack_bf16x2(fmaf(y0, t.x, x0 * t.y), fmaf(y1, t.z, x1 * t.w));
   }
   *pa = A;
   *pb = Bv;
@@ -232,8 +234,8 @@ __device__ __forceinline__ void rotate_q_row_scalar(uint8_t* tile, int row, int 
     uint16_t* pa = reinterpret_cast<uint16_t*>(tile + oa);
     uint16_t* pb = reinterpret_cast<uint16_t*>(tile + ob);
     const float x = __uint_as_float((uint32_t)*pa << 16), y = __uint_as_float((uint32_t)*pb << 16);
-    *pa = __bfloat16_as_ushort(__float2bfloat16_rn(x * c.x - y * c.y));
-    *pb = __bfloat16_as_ushort(__float2bfloat16_rn(y * c.x + x * c.y));
+    *pa = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(x, c.x, -(y * c.y))));
+    *pb = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(y, c.x, x * c.y)));
   }
 }
 

@@ -133,6 +133,26 @@ def test_score_extremes(cuda_device, kind, W, theta):
     check_no_device_error()
 
 
+@pytest.mark.parametrize("W,theta,r,table", [(200, 1e4, 128, False), (-1, 5e6, 64, False), (-1, 5e6, 64, True),
+                                             (96, 5e5, 24, False)])
+def test_in_kernel_rotation_equals_rope_qk_bitwise(cuda_device, W, theta, r, table):
+    """The in-kernel Q rotation and the key pre-pass round exactly as
+    swa_rope_qk does: prefill with RoPE equals, bit for bit, prefill without
+    rotation on q and k rotated beforehand by swa_rope_qk."""
+    B, S, Hq, Hkv = 2, 333, 8, 2
+    freq = scaled_inv_freq(theta, r) if table else None
+    p = api.LayerParams(Hq, Hkv, 128, W, theta, r, inv_freq=freq)
+    plain = api.LayerParams(Hq, Hkv, 128, W, 0.0, r)
+    d = {k: t.to(cuda_device) for k, t in inputs.prefill_inputs(B, S, Hq, Hkv, 128, 780 + r).items()}
+    out = api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"])
+    q, k = d["q"].clone(), d["k"].clone()
+    api.rope_qk(p, q=q, k=k)
+    out_pre = api.attn_prefill(plain, q, k, d["v"], d["gate"])
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), out_pre.view(torch.int16))
+    check_no_device_error()
+
+
 def test_saturated_gate_logits(cuda_device):
     """Gate logits of +-60 and +-1e4 saturate the sigmoid: the output is the
     ungated attention, about 1e-26 of it (sigmoid(-60)), or exactly zero
