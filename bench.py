@@ -118,6 +118,11 @@ def measured_prefill_traffic(workload: str):
     return None
 
 
+# B200 spec sheet (dense, no sparsity) figures, reported beside the measured
+# peaks: bf16 tensor 2.25 PFLOP/s; HBM3e 7.7 TB/s (HGX board figure)
+SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 7700.0}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -606,6 +611,7 @@ def main():
             "clocks": clocks, "gpu_launches": launches}
     line["roofline"] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                         "frac": achieved / peaks["bf16_tflops"], "traffic": measured_prefill_traffic(c.name),
+                        "frac_of_spec": achieved / SPEC_PEAKS["bf16_tflops"],
                         "peak_source": f"{peak_src} bf16 burst",
                         "kernel": "swa_attn_prefill (key-RoPE pre-pass + attention kernel), CUDA events"}
     if not args.no_e2e:
@@ -627,6 +633,7 @@ def main():
                 c_ms = bench_prefill_chunk(cc, 20 if cc.window > 0 else 5, 3, dev)
                 tf = chunk_flops(cc) / (c_ms / 1e3) / 1e12
                 chunks[cc.name] = {"ms": c_ms, "TFLOP/s": tf, "frac_bf16": tf / peaks["bf16_tflops"],
+                                   "frac_of_spec": tf / SPEC_PEAKS["bf16_tflops"],
                                    "peak_source": f"{peak_src} bf16 burst"}
             extra, mqs = {}, {}
             for kind, dc in (("decode", configs.DECODE_SLIDING), ("mq", configs.MQ_SLIDING),
@@ -637,6 +644,7 @@ def main():
                 (extra if kind == "decode" else mqs)[dc.name] = {
                     "ms": d_ms, "ms_eager": e_ms, "timing": "CUDA graph replay of the steps (ms_eager: launched one by one)",
                     "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                    "frac_of_spec": gbs / SPEC_PEAKS["hbm_gbs"],
                     "peak_source": f"{peak_src} hbm copy"}
             line["decode"] = extra
             line["decode_mq"] = mqs
