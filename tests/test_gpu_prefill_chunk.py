@@ -1,14 +1,16 @@
 """swa_attn_prefill_chunk on the GPU: a sequence prefilled in several chunks
 against the KV cache gives the rows of the whole-sequence attention the
 oracle computes, and leaves the cache exactly as appending every token with
-swa_rope_qk would (ring: the last W positions; linear: all of them)."""
+swa_rope_qk would (ring: the last W positions; linear: all of them); the
+bench's two continued-prefill workloads at full size on seeded rows."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from full_gqa_attention_swa_b200 import api, inputs
-from gpu_helpers import assert_close, bits, check_no_device_error, oracle_layer, scaled_inv_freq
+from full_gqa_attention_swa_b200 import api, configs, inputs
+from gpu_helpers import (assert_close, bits, check_no_device_error, oracle_layer, prefill_rows_sample,
+                         scaled_inv_freq)
 
 pytestmark = pytest.mark.gpu
 
@@ -104,4 +106,31 @@ def test_decode_after_chunked_prefill(cuda_device, p, C):
     out = api.attn_decode(p, q[:, 0].contiguous(), d["gate"][:, L - 1].to(cuda_device).contiguous(), kc, vc, lens, L)
     torch.cuda.synchronize()
     assert_close(out.reshape(B * 8, 128), ref.reshape(B * 8, 128), "decode after chunks")
+    check_no_device_error()
+
+
+@pytest.mark.parametrize("cc", [configs.CHUNK_SLIDING, configs.CHUNK_FULL], ids=lambda c: c.name)
+def test_bench_chunk_workloads_sampled(cuda_device, cc):
+    """The continued-prefill workloads the bench times, at full size: the
+    history (positions < pos0) is appended to a fresh cache the way a
+    caller's earlier steps would (swa_rope_qk), the chunk then runs as in the
+    bench, and seeded rows of it (first, last, band and tile edges, random,
+    every head) match the oracle's whole-sequence prefill."""
+    p = api.LayerParams(cc.Hq, cc.Hkv, 128, cc.window, cc.theta, cc.rotary_dim)
+    L = cc.pos0 + cc.S
+    d = inputs.prefill_inputs(cc.B, L, cc.Hq, cc.Hkv, 128, cc.seed)
+    C = cc.window if cc.window > 0 else L
+    kc = torch.zeros(cc.B, cc.Hkv, C, 128, dtype=torch.bfloat16, device=cuda_device)
+    vc = torch.zeros_like(kc)
+    hist, new = slice(0, cc.pos0), slice(cc.pos0, L)
+    api.rope_qk(p, k=d["k"][:, hist].to(cuda_device).contiguous(), pos0=0,
+                v=d["v"][:, hist].to(cuda_device).contiguous(), k_cache=kc, v_cache=vc)
+    dev = {k: t[:, new].to(cuda_device).contiguous() for k, t in d.items()}
+    out = api.attn_prefill_chunk(p, cc.pos0, dev["q"], dev["k"], dev["v"], dev["gate"], kc, vc)
+    torch.cuda.synchronize()
+    rows = prefill_rows_sample(cc.B, cc.S, cc.Hq, cc.window, seed=cc.seed, n_random=48)
+    rows[:, 1] += cc.pos0                     # positions of the chunk's rows in the whole sequence
+    ref = oracle.prefill(oracle_layer(p), bits(d["q"]), bits(d["k"]), bits(d["v"]), d["gate"].numpy(), rows=rows)
+    idx = [torch.from_numpy(rows[:, 0]), torch.from_numpy(rows[:, 1] - cc.pos0), torch.from_numpy(rows[:, 2])]
+    assert_close(out.cpu()[idx[0], idx[1], idx[2]], ref, cc.name)
     check_no_device_error()
