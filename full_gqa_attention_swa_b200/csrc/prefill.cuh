@@ -412,14 +412,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint64_t kd = kdesc0 + (uint64_t)(((ki % NK) * kTileBytes) >> 4);
-            // unrolled by 2: fewer loop instructions between MMAs on the issuer's
-            // busy sub-partition (C2 -1.7 %, C3 -2.9 %; fully unrolled it spills
-            // at this warp's 56 registers, by 4 it ran slower)
+            // unrolled by 2, descriptors advanced in their low words: fewer
+            // instructions between MMAs on the issuer's busy sub-partition (C2
+            // -1.7 % and -2.2 %, C3 -2.9 % and -2.1 %; fully unrolled it spills at
+            // this warp's 56 registers, by 4 it ran slower)
 #pragma unroll 2
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t off = (uint64_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
-              umma_ss(tmem, qd0 + off, kd + off, idesc_qk, kk > 0);
-              umma_ss(tmem + 128, qd1 + off, kd + off, idesc_qk, kk > 0);
+              const uint32_t o32 = (uint32_t)off;
+              umma_ss_lh(tmem, (uint32_t)qd0 + o32, (uint32_t)(qd0 >> 32), (uint32_t)kd + o32, (uint32_t)(kd >> 32),
+                         idesc_qk, kk > 0);
+              umma_ss_lh(tmem + 128, (uint32_t)qd1 + o32, (uint32_t)(qd1 >> 32), (uint32_t)kd + o32,
+                         (uint32_t)(kd >> 32), idesc_qk, kk > 0);
             }
             umma_commit(&sm.s_full);
             umma_commit(&sm.k_empty[ki % NK]);
@@ -442,8 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t aoff = (uint64_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
               const uint64_t boff = (uint64_t)((kk * 2048) >> 4);
               const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-              umma_ss(tmem + 256, pd0 + aoff, vd + boff, idesc_pv, acc);
-              umma_ss(tmem + 384, pd1 + aoff, vd + boff, idesc_pv, acc);
+              umma_ss_lh(tmem + 256, (uint32_t)pd0 + (uint32_t)aoff, (uint32_t)(pd0 >> 32), (uint32_t)vd + (uint32_t)boff,
+                         (uint32_t)(vd >> 32), idesc_pv, acc);
+              umma_ss_lh(tmem + 384, (uint32_t)pd1 + (uint32_t)aoff, (uint32_t)(pd1 >> 32), (uint32_t)vd + (uint32_t)boff,
+                         (uint32_t)(vd >> 32), idesc_pv, acc);
             }
             umma_commit(&sm.pv_done);
             umma_commit(&sm.v_empty[vi % NV]);
