@@ -2,14 +2,20 @@
 core on B200, as a fraction of the measured peaks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload NAME] [--no-decode]
+                    [--workload NAME] [--no-decode] [--only LEG]
 
 One step = one swa_attn_prefill call (RoPE of the keys, then the fused
-tcgen05 attention kernel with RoPE on the Q tile load, banded causal mask,
-online softmax, P.V and the head gate) over one batch of the Step-3.7-Flash
-sliding-layer workload (B1 S8192 Hq96 Hkv8 W512, theta 1e4).  Inputs are
-resident in HBM and rotate over 4 copies of 439 MB each (more than the
-126 MB L2), so no step reads the previous step's data from L2.
+tcgen05 attention kernel with RoPE on the Q tile load, causal mask, online
+softmax, P.V and the head gate) over one batch of the largest single-GPU
+workload, the Step-3.7-Flash full-attention layer (B1 S32768 Hq64 Hkv8,
+causal, theta 5e6 on the first 64 dims).  Inputs are resident in HBM and
+rotate over 4 copies (1.2 GB each, far more than the 126 MB L2), so no step
+reads the previous step's data from L2.
+
+Beside the headline, the same line carries the other three prefill
+workloads (the Step sliding layer and the Muse sliding / full layers), each
+timed the same way, and the decode, multi-query decode and continued-prefill
+legs.
 
 With torchrun (N > 1) every rank runs the same workload on its own GPU (the
 work shards by sequence / kv-head with no exchange; weak scaling); time is
@@ -90,15 +96,16 @@ def decode_mq_bytes(c, lens) -> int:
     return keys * c.Hkv * 128 * 2 * 2 + c.B * c.T * (c.Hq * (128 * 2 * 2 + 4) + c.Hkv * 128 * 2 * 2)
 
 
-# DRAM traffic per launch of the prefill attention kernel from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/prefill_kernel_step37_sliding.md).
-# It describes only the kernel source it was taken on, so it is reported only
-# while csrc/prefill.cuh still hashes to the recorded digest, else null.
+# DRAM traffic per launch of the prefill attention kernel from ncu captures
+# (dram__bytes_read.sum + dram__bytes_write.sum, one launch per workload; the
+# summaries under profiles/).  A figure describes only the kernel source it was
+# taken on, so it is reported only while csrc/prefill.cuh and csrc/ptx.cuh still
+# hash to the recorded digest, else null.
 PREFILL_TRAFFIC = {
-    "workload": "step37_sliding_B1_S8192_Hq96_Hkv8_W512",
-    "bytes": 401.0e6,
-    # prefill.cuh and ptx.cuh (the kernel and its PTX helpers) as captured; any change makes the figure stale
+    # prefill.cuh and ptx.cuh as captured; any change makes the figures stale
     "source_sha256": "57ed7ab024c3695d70695ef0194643a9b44636be3ca9f762ab7f3719c94f8534",
+    "bytes": {"step37_sliding_B1_S8192_Hq96_Hkv8_W512": 401.0e6,
+              "step37_full_B1_S32768_Hq64_Hkv8_causal": 4262.8e6},
 }
 PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh")
 
@@ -113,8 +120,8 @@ def prefill_source_digest():
 
 
 def measured_prefill_traffic(workload: str):
-    if workload == PREFILL_TRAFFIC["workload"] and prefill_source_digest() == PREFILL_TRAFFIC["source_sha256"]:
-        return PREFILL_TRAFFIC["bytes"]
+    if workload in PREFILL_TRAFFIC["bytes"] and prefill_source_digest() == PREFILL_TRAFFIC["source_sha256"]:
+        return PREFILL_TRAFFIC["bytes"][workload]
     return None
 
 
@@ -163,6 +170,9 @@ class ClockSampler:
         self.period = period_s
         self._stop = threading.Event()
         self._thread = None
+        self.nv = None
+        if index < 0:
+            return
         try:
             import pynvml
 
@@ -217,19 +227,19 @@ def _layer(c):
     return api.LayerParams(c.Hq, c.Hkv, 128, c.window, c.theta, c.rotary_dim)
 
 
-def bench_prefill(c, steps: int, warmup: int, dev, dist=None):
+def bench_prefill(c, steps: int, warmup: int, dev, dist=None, n_rotate: int = N_ROTATE, clocks_on: bool = True):
     from full_gqa_attention_swa_b200 import api
 
     p = _layer(c)
     sets = [inputs.prefill_inputs(c.B, c.S, c.Hq, c.Hkv, 128, c.seed + 17 * r, device=dev)
-            for r in range(N_ROTATE)]
+            for r in range(n_rotate)]
     out = torch.empty(c.B, c.S, c.Hq, 128, dtype=torch.bfloat16, device=dev)
     ws_bytes = api.prefill_workspace_size(p, c.B, c.S)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
-        d = sets[i % N_ROTATE]
+        d = sets[i % n_rotate]
         api.attn_prefill(p, d["q"], d["k"], d["v"], d["gate"], out=out, workspace=ws, stream=stream)
 
     for i in range(max(warmup, 0)):
@@ -239,7 +249,7 @@ def bench_prefill(c, steps: int, warmup: int, dev, dist=None):
         dist.barrier()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clocks:
+    with ClockSampler(dev.index if clocks_on else -1) as clocks:
         torch.cuda.synchronize(dev)
         ev0.record(stream)
         for i in range(steps):
@@ -250,6 +260,8 @@ def bench_prefill(c, steps: int, warmup: int, dev, dist=None):
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
     launches = steps * (2 if ws_bytes > 0 else 1)
+    del sets
+    torch.cuda.empty_cache()
     return ms, clocks.summary(), launches
 
 
@@ -499,12 +511,16 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
-    ap.add_argument("--workload", default=configs.STEP_SLIDING.name, choices=sorted(configs.PREFILL))
+    ap.add_argument("--workload", default=configs.STEP_FULL.name, choices=sorted(configs.PREFILL))
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--only", choices=["all", "prefill", "decode_sliding", "decode_full", "chunk_sliding",
                                        "chunk_full", "decode_mq_sliding", "decode_mq_full"], default="all",
                     help="run one leg only (profiling); prints that leg's own JSON line")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--rotate", type=int, default=N_ROTATE,
+                    help="input sets the prefill steps rotate over (fewer: a smaller device footprint, for profiling)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="with --only decode_*: run that layer with this many sequences (profiling a capped case)")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     c = configs.PREFILL[args.workload]
@@ -515,7 +531,7 @@ def main():
     cfg = {"workload": c.name, "global_batch": c.B * world, "seq_len": c.S, "q_heads": c.Hq, "kv_heads": c.Hkv,
            "head_dim": 128, "window": c.window, "rope_theta": c.theta, "rotary_dim": c.rotary_dim,
            "parallelism": f"replicas{world}" if world > 1 else "single",
-           "l2": f"rotating {N_ROTATE} input sets of {prefill_bytes(c) / 1e6:.0f} MB (> 126 MB L2)"}
+           "l2": f"rotating {max(args.rotate, 1)} input sets of {prefill_bytes(c) / 1e6:.0f} MB (> 126 MB L2)"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -579,6 +595,10 @@ def main():
             dc = configs.MQ_SLIDING if args.only == "decode_mq_sliding" else configs.MQ_FULL
         else:
             dc = configs.DECODE_SLIDING if args.only == "decode_sliding" else configs.DECODE_FULL
+        if args.decode_batch > 0:
+            import dataclasses
+
+            dc = dataclasses.replace(dc, B=args.decode_batch, name=f"{dc.name}_capped_B{args.decode_batch}")
         if dist is not None:
             dist.barrier()
         run = bench_decode_mq if mq else bench_decode
@@ -597,7 +617,7 @@ def main():
             dist.destroy_process_group()
         return
 
-    ms, clocks, launches = bench_prefill(c, args.steps, max(args.warmup, 3), dev, dist)
+    ms, clocks, launches = bench_prefill(c, args.steps, max(args.warmup, 3), dev, dist, n_rotate=max(args.rotate, 1))
     ms = max_over_ranks(ms, dist, dev)
     value, _ = combine_ranks([ms], world, flops * args.steps / 1e12)   # TFLOP/s over all ranks
     per_step_ms = ms / args.steps
@@ -626,6 +646,24 @@ def main():
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     if rank == 0:
         # the extra legs and the CPU baseline describe one GPU: single-process runs only
+        if world == 1 and args.only == "all":
+            # the other prefill workloads, each timed like the headline
+            # (rotating input sets, CUDA events around the steps)
+            legs = {}
+            for pc in (configs.STEP_SLIDING, configs.STEP_FULL, configs.MUSE_SLIDING, configs.MUSE_FULL):
+                if pc.name == c.name:
+                    p_ms, p_steps = ms, args.steps
+                else:
+                    p_steps = max(5, min(200, int(200.0 / max(prefill_flops(pc) / 1e12, 1e-3))))
+                    p_ms, _, _ = bench_prefill(pc, p_steps, 3, dev, n_rotate=max(args.rotate, 1), clocks_on=False)
+                tf = prefill_flops(pc) / (p_ms / p_steps / 1e3) / 1e12
+                legs[pc.name] = {"ms": p_ms / p_steps, "steps": p_steps, "TFLOP/s": tf,
+                                 "frac_bf16": tf / peaks["bf16_tflops"], "frac_of_spec": tf / SPEC_PEAKS["bf16_tflops"],
+                                 "peak_source": f"{peak_src} bf16 burst", "unmasked_flop": prefill_flops(pc),
+                                 "traffic": measured_prefill_traffic(pc.name),
+                                 "timing": "swa_attn_prefill (key pre-pass + attention), CUDA events"}
+            line["prefill"] = legs
+            assert api.device_error() == 0, "a kernel reported a bounded-wait timeout"
         if world == 1 and not args.no_decode and args.only == "all":
             # the short legs first, the two 34 GB full-layer decode legs last
             chunks = {}
