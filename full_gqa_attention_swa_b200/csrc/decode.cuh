@@ -90,6 +90,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_split_kernel(cons
   const int L = a.seq_lens[b];
   const int n_vis = (a.window > 0 && L > a.window) ? a.window : L;
   const int k_begin = split * a.chunk;
+  // a length beyond the host's max_len breaks the call's contract: the keys
+  // past the planned splits are not read, and the error word says so
+  if (threadIdx.x == 0 && kvh == 0 && split == a.max_splits - 1 && n_vis > k_begin + a.chunk)
+    record_error(kErrDecode + 3);
   if (L < 1 || k_begin >= n_vis) return;  // uniform over the CTA, before any barrier
   const int k_end = min(n_vis, k_begin + a.chunk);
   const int n_blocks = (k_end - k_begin + KB - 1) / KB;
@@ -326,7 +330,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a)
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int L = a.seq_lens[b];
   const int n_vis = (a.window > 0 && L > a.window) ? a.window : L;
-  const int n_split = (n_vis + a.chunk - 1) / a.chunk;
+  // never past this row's planned partials (a length beyond max_len is
+  // recorded by the split kernel)
+  const int n_split = min((n_vis + a.chunk - 1) / a.chunk, a.max_splits);
   const size_t base = ((size_t)b * a.Hq + h) * a.max_splits;
   float M = -INFINITY;
   for (int s = 0; s < n_split; ++s) M = fmaxf(M, a.part_ml[base + s].x);

@@ -287,34 +287,30 @@ swa_status scratch_for_current_device(void** ptr) {
 }
 
 // The usual decode plan, or -- when its partials exceed the static array --
-// the same work in fewer, longer splits.
-swa_status plan_decode_no_alloc(const swa_layer_params* p, int B, int max_len, DecodePlan* out) {
+// the same work in fewer, longer splits, down to one split per row, which
+// writes the output directly and needs no scratch at all.
+DecodePlan plan_decode_no_alloc(const swa_layer_params* p, int B, int max_len) {
   DecodePlan pl = plan_decode(p, B, max_len);
-  if (pl.total <= SWA_NO_ALLOC_SCRATCH_BYTES) {
-    *out = pl;
-    return SWA_OK;
-  }
+  if (pl.total <= SWA_NO_ALLOC_SCRATCH_BYTES) return pl;
   const long long kb = swa::kDecodeKeyBlock;
   const long long n_vis = p->window > 0 ? (max_len < p->window ? max_len : p->window) : max_len;
   const size_t rows = (size_t)B * p->num_q_heads;
   const size_t per_split = rows * (kHeadDim * sizeof(float) + sizeof(float2));
   // two 256-byte alignment pads between and after the two arrays
-  long long fit = (long long)((SWA_NO_ALLOC_SCRATCH_BYTES - 512) / per_split);
-  for (; fit >= 2; --fit) {
+  for (long long fit = (long long)((SWA_NO_ALLOC_SCRATCH_BYTES - 512) / per_split); fit >= 2; --fit) {
     DecodePlan q{};
     q.chunk = (int)(((n_vis + fit - 1) / fit + kb - 1) / kb * kb);
     q.splits = (int)((n_vis + q.chunk - 1) / q.chunk);
+    if (q.splits < 2) break;
     q.o_bytes = round_up(rows * q.splits * kHeadDim * sizeof(float), 256);
     q.ml_bytes = round_up(rows * q.splits * sizeof(float2), 256);
     q.total = q.o_bytes + q.ml_bytes;
-    if (q.total <= SWA_NO_ALLOC_SCRATCH_BYTES) {
-      *out = q;
-      return SWA_OK;
-    }
+    if (q.total <= SWA_NO_ALLOC_SCRATCH_BYTES) return q;
   }
-  return fail(SWA_ERR_UNSUPPORTED,
-              "no-alloc decode: %zu q-head rows need %zu bytes per split; the static scratch holds %u bytes",
-              rows, per_split, (unsigned)SWA_NO_ALLOC_SCRATCH_BYTES);
+  DecodePlan one{};
+  one.chunk = (int)((n_vis + kb - 1) / kb * kb);
+  one.splits = 1;
+  return one;
 }
 
 }  // namespace
@@ -672,10 +668,11 @@ swa_status swa_attn_decode_no_alloc(const swa_layer_params* p, int32_t B, const 
   if (p->window < 0 && max_len > cache_capacity)
     return fail(SWA_ERR_INVALID_ARG, "full layer: max_len=%d exceeds cache_capacity=%d", max_len, cache_capacity);
   if (B > 65535 || Hkv > 65535) return fail(SWA_ERR_UNSUPPORTED, "B=%d or Hkv=%d too large (grid y / z)", B, Hkv);
-  DecodePlan pl;
-  if ((st = plan_decode_no_alloc(p, B, max_len, &pl)) != SWA_OK) return st;
+  // the one-time address lookup runs on the first call on a device, whatever
+  // that call's plan
   void* scratch = nullptr;
-  if (pl.splits > 1 && (st = scratch_for_current_device(&scratch)) != SWA_OK) return st;
+  if ((st = scratch_for_current_device(&scratch)) != SWA_OK) return st;
+  const DecodePlan pl = plan_decode_no_alloc(p, B, max_len);
   CUtensorMap km, vm;
   if ((st = encode_cache(&km, k_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
   if ((st = encode_cache(&vm, v_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;

@@ -206,7 +206,10 @@ SWA_API size_t swa_decode_workspace_size(const swa_layer_params* params, int32_t
  *   seq_lens [B] int32 device, 1 <= L_b, counting the current token (already
  *            appended); the query sits at position L_b - 1 and sees the
  *            min(L_b, W) filled ring slots (sliding) or slots 0..L_b-1 (full).
- *   max_len  host-side upper bound of seq_lens (sizes the split grid).
+ *   max_len  host-side upper bound of seq_lens (sizes the split grid).  A
+ *            sequence longer than max_len breaks this contract: the keys
+ *            past the planned splits are not read (its output is wrong) and
+ *            device error 203 is recorded; no read leaves the workspace.
  *   out      [B, Hq, D] bf16
  *   workspace / workspace_bytes: at least swa_decode_workspace_size() bytes
  *            (may be NULL when that is 0); overwritten.
@@ -311,10 +314,11 @@ SWA_API const char* swa_version(void);
  * (sequence, q-head) row takes 520 bytes there.  When the usual split of the
  * cache would not fit, fewer, longer splits are used; when even two splits
  * per row do not fit (B * Hq * 2 * 520 bytes, plus 512 bytes of alignment,
- * above SWA_NO_ALLOC_SCRATCH_BYTES) and the sequences need splitting, the call
- * returns SWA_ERR_UNSUPPORTED and launches nothing.  Nothing in the array
- * needs to start at zero: every partial a call reads was written earlier in
- * the same call.
+ * above SWA_NO_ALLOC_SCRATCH_BYTES), each row's whole visible range runs as
+ * one split, which writes the output directly and uses none of the array
+ * (slower for long contexts and small batches, never refused for size).
+ * Nothing in the array needs to start at zero: every partial a call reads was
+ * written earlier in the same call.
  *
  * All calls on a device share that array, and it keeps the contents of the
  * last call: two calls whose kernels overlap on the GPU (different streams,

@@ -133,6 +133,36 @@ def test_decode_argument_errors(lib):
     assert lib.swa_attn_decode(sl, 70000, *args(512, 512)) == 2          # B beyond the grid's z limit
 
 
+def test_decode_no_alloc_argument_errors(lib):
+    """The no-alloc decode's host checks, which all run before it touches the
+    device (no GPU needed): the same rules as swa_attn_decode, with out
+    required."""
+    sl = _P(num_q_heads=96, num_kv_heads=8, window=512)
+    full = _P(num_q_heads=64, num_kv_heads=8, window=-1, rope_theta=5e6, rotary_dim=64)
+    # (q, gate, k_cache, v_cache, C, seq_lens, max_len, out, stream)
+    args = lambda C, max_len: [FAKE, NULL, FAKE, FAKE, C, FAKE, max_len, FAKE, NULL]
+    f = lib.swa_attn_decode_no_alloc
+    assert f(sl, 4, *args(256, 100)) == 1                                # ring capacity != W
+    assert f(full, 4, *args(1000, 2000)) == 1                            # max_len > capacity
+    assert f(full, 4, *args(1000, 0)) == 1                               # max_len < 1
+    assert f(full, 4, *args(0, 10)) == 1                                 # capacity < 1
+    assert f(_P(num_q_heads=34, num_kv_heads=2), 4, *args(64, 10)) == 2  # G > 16
+    assert f(sl, 70000, *args(512, 512)) == 2                            # B beyond the grid's z limit
+    assert f(sl, -1, *args(512, 512)) == 1                               # negative batch
+    assert f(sl, 0, *args(512, 512)) == 0                                # empty batch: nothing launched
+    assert f(None, 4, *args(512, 512)) == 1                              # no parameters
+    for i, name in ((0, "q"), (2, "k_cache"), (3, "v_cache"), (5, "seq_lens"), (7, "out")):
+        a = args(512, 512)
+        a[i] = NULL
+        assert f(sl, 4, *a) == 1, name                                   # required pointer missing
+        a[i] = MIS
+        assert f(sl, 4, *a) == 1, name                                   # misaligned pointer
+    a = args(512, 512)
+    a[1] = MIS
+    assert f(sl, 4, *a) == 1                                             # misaligned gate
+    assert b"aligned" in lib.swa_last_error_detail()
+
+
 def test_rope_argument_errors(lib):
     p = _P(window=16)
     assert lib.swa_rope_qk(p, 2, 4, FAKE, FAKE, NULL, 0, FAKE, FAKE, NULL, 16, NULL) == 1   # one cache only

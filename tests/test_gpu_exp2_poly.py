@@ -22,7 +22,7 @@ REL_BOUND = 1.1e-4
 
 
 def test_header_coefficients_match_fit():
-    out = subprocess.run([sys.executable, os.path.join(CSRC, "exp2_poly_fit.py")], capture_output=True, text=True,
+    out = subprocess.run([sys.executable, os.path.join(REPO, "tests", "exp2_poly_fit.py")], capture_output=True, text=True,
                          check=True).stdout
     fitted = [float(v) for v in re.findall(r"c\d = ([-0-9.e+]+)f", out)]
     assert len(fitted) == 3

@@ -86,7 +86,6 @@ def test_no_gate_and_custom_scale(cuda_device):
     check_no_device_error()
 
 
-@pytest.mark.slow
 def _score_extreme_inputs(kind, B, S, Hq, Hkv, seed):
     """Inputs whose scores stress the online softmax.  'large': q and k times
     3, so scores have a standard deviation near 9 (natural units) and a few
