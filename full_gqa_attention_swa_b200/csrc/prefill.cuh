@@ -1,7 +1,6 @@
 // Prefill attention on sm_100a: RoPE'd Q, banded causal mask, GQA, online
 // softmax, P.V and the per-head sigmoid gate, with tcgen05 tensor-core MMAs
-// accumulating in tensor memory, TMA loads into shared memory and a TMA
-// store of the output.
+// accumulating in tensor memory and TMA loads into shared memory.
 //
 // Follows the "Step-3.7-Flash-oQ3e" explainer: section 2.2 (sliding-window
 // causal mask of W keys on sliding layers, plain causal mask on full layers)
@@ -9,46 +8,40 @@
 // gate); the "Step-3.7-Flash" spec card's GQA groups; the "Muse-Glimmer-30B-
 // 6bit" explainer's theta = 0 (no rotation) on full layers.
 //
-// Work unit ("tile"): 128 query rows x two q-heads of the same kv-head, so
-// every K/V tile in shared memory feeds two 128x128 score tiles.  Query row r
-// sits at key-space position i = q_off + r (q_off > 0 when a chunk of queries
-// continues a sequence whose earlier keys are in the K/V source).  A tile
-// loops over the key tiles of its band [i0 - W + 1, i0 + 127]; key tiles
-// wholly outside the band are never loaded, and the mask is evaluated only
-// on tiles the band edge or the diagonal cuts.  The grid is persistent (one
-// CTA per SM); a CTA walks tiles blockIdx.x, +gridDim.x, ... in an order
-// that puts the longest (latest-row) tiles first.  Loads, rotation and the
-// output store of neighbouring tiles overlap with the tensor-core work.
+// Work unit ("tile"): 128 query rows x two q-heads ("head slots") of the same
+// kv-head, so every K/V tile in shared memory feeds two 128x128 score tiles.
+// Query row r sits at key-space position i = q_off + r.  A tile loops over
+// the key tiles of its band [i0 - W + 1, i0 + 127]; key tiles wholly outside
+// the band are never loaded, and the mask is evaluated only on tiles the band
+// edge or the diagonal cuts.  The grid is persistent (one CTA per SM); a CTA
+// walks tiles blockIdx.x, +gridDim.x, ... with the longest (latest-row) tiles
+// first.
+//
+// Pipeline.  P (bf16) is written by the softmax into the tensor-memory
+// columns of the S tile it came from, and P.V reads it from there (A operand
+// in tensor memory), so no shared memory holds P.  That leaves room for two
+// Q buffers per head slot: the next tile's Q is loaded and rotated while the
+// current tile runs, and the first QK^T of the next tile follows the last P.V
+// of this one without a gap.  The tensor pipe runs, per head slot s and key
+// tile j, the block [O_s += P_s(j) V(j); S_s = Q_s K(j+1)^T], the two slots'
+// blocks alternating, so one slot's softmax overlaps the other slot's MMAs.
+// The MMAs of one thread execute in issue order, so S_s(j+1) overwrites the
+// columns of P_s(j) only after P_s(j).V has read them.
 //
 // Warp roles (16 warps, registers rebalanced with setmaxnreg):
-//   warps 0-3   head slot 0: Q rotation, softmax (thread = query row)
-//   warps 4-7   head slot 1: same
-//   warps 8-11  O rescaling ("correction") and the epilogue (O/l * gate ->
-//               bf16 -> the slot's P buffer in shared memory)
+//   warps 0-3   head slot 0 softmax (thread = query row); rescales its own
+//               O row when the running max moves (rare: lazy threshold)
+//   warps 4-7   head slot 1 softmax
+//   warps 8-11  next tile's Q rotation, then this tile's epilogue
+//               (O / l * sigmoid(gate) -> bf16 -> global, thread = row)
 //   warp 12     tcgen05.mma issuer (one thread)
-//   warp 13     TMA producer (one thread)
-//   warp 14     TMA store of the output tiles (one thread)
-//   warp 15     folds K / V arrivals into the issuer's barriers (one thread)
-// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384)
-// O1 [384,512).  P (bf16) goes to a shared-memory buffer per head slot.
-//
-// Per key tile j and head slot s:
-//   MMA:     S_s = Q_s K_j^T            -> s_full (both slots)
-//   softmax: read S_s                   -> s_free (both slots: S(j+1) may start)
-//            m, alpha                   -> alpha_full[s]
-//            P_s = 2^(S_s - m) -> smem  -> pv_ready
-//   correct: wait PV_s(j-1), O_s *= alpha (skipped when alpha == 1 for the
-//            whole warp)                -> pv_ready
-//   MMA:     O_s += P_s V_j             -> pv_done (both slots; frees the P buffers)
-// The MMA thread waits on one barrier per hand-off (s_free, pv_ready) rather
-// than one per slot and producer: each wait is a shared-memory round trip that
-// queues behind the softmax warps' SFU traffic on the same sub-partition.  A
-// helper thread folds the K / V tile arrivals into those two barriers.
-// The exponentials run on the SFU (a polynomial path on the FMA pipe exists,
-// see poly_column_pair).
+//   warp 13     K / V TMA producer (one thread), three-stage ring
+//   warp 15     Q TMA producer (one thread)
+// Tensor memory (512 columns): S0/P0 [0,128) S1/P1 [128,256) O0 [256,384)
+// O1 [384,512).
 // The max used for the exponentials only moves when the new row max exceeds
-// it by more than 8 (log2 units), so most tiles need no O rescale; exp2 of a
-// score then stays below 2^8, and the final normalisation by the row sum
+// it by more than 8 (log2 units), so most key tiles need no O rescale; exp2
+// of a score then stays below 2^8, and the final normalisation by the row sum
 // computed with the same max is exact.
 #pragma once
 #include "swa_internal.cuh"
@@ -59,8 +52,7 @@ namespace prefill_detail {
 
 constexpr int BM = 128;                         // query rows per tile
 constexpr int BN = 128;                         // keys per key tile
-constexpr int NK = 2;                           // K tile ring
-constexpr int NV = 1;                           // V tile ring
+constexpr int kKvStages = 3;                    // K / V ring (loads K0 V0 K1 V1 ...)
 constexpr int kThreads = 512;
 constexpr uint32_t kBoxBytes = 128 * 128;       // 128 rows x 64 bf16
 constexpr uint32_t kTileBytes = 2 * kBoxBytes;  // 128 rows x 128 bf16
@@ -75,26 +67,19 @@ constexpr uint32_t kRegsOther = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
 
-// 231,712 bytes: within the 232,448-byte opt-in limit only because the
-// dynamic shared memory window starts 1024-byte aligned (checked at entry).
-struct PrefillSmem {
-  uint8_t q[2][kTileBytes];    // Q of each head slot (rotated in place)
-  uint8_t p[2][kTileBytes];    // P (bf16) of each slot; also stages its output tile
-  uint8_t k[NK][kTileBytes];
-  uint8_t v[NV][kTileBytes];
-  float alpha[2][BM];
-  float lsum[2][BM];
-  uint64_t q_full[2], q_empty[2];
-  uint64_t q_ready;  // both slots' Q rotated (256 arrivals)
-  uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
-  uint64_t alpha_full[2], alpha_empty[2];
-  uint64_t s_full;    // S of both slots complete
-  uint64_t pv_done;   // P.V of both slots complete (frees both P buffers)
-  uint64_t s_free;    // both slots have read S, and the next K tile has landed (256 + 1 arrivals)
-  uint64_t pv_ready;  // both slots' P written and O rescaled, and the V tile has landed (512 + 1)
-  uint64_t l_full[2], l_empty[2];
-  uint64_t ost_full[2];  // output tile staged in p[s]
-  uint64_t pfree[2];     // the store of that tile has read p[s]
+struct Smem {
+  uint8_t q[2][2][kTileBytes];     // [tile parity][head slot]: Q, rotated in place
+  uint8_t kv[kKvStages][kTileBytes];
+  float lsum[2][2][BM];            // [tile parity][head slot][row]: softmax row sums
+  uint64_t q_full[2][2];           // Q of [parity][slot] landed
+  uint64_t q_empty[2][2];          // the last QK^T reading Q[parity][slot] completed
+  uint64_t q_ready[2];             // both slots' Q rotated (128 arrivals)
+  uint64_t kv_full[kKvStages], kv_empty[kKvStages];
+  uint64_t s_full[2];              // S_s complete (and every earlier MMA, P_s.V included)
+  uint64_t p_full[2];              // P_s written, O_s rescaled (128 arrivals)
+  uint64_t o_done[2];              // the tile's last P_s.V complete
+  uint64_t o_free[2];              // the epilogue has read O_s (128 arrivals)
+  uint64_t l_full[2][2];           // [parity][slot] row sums written (128 arrivals)
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -136,14 +121,6 @@ __device__ __forceinline__ Tile decode_tile(const PrefillArgs& a, int t) {
   return T;
 }
 
-// Column pairs (of every 8) whose exponentials run on the FMA pipe
-// (exp2_poly2) instead of the SFU.  Zero: the step is bound by the tensor
-// pipe and the MMA thread's hand-offs, not by the SFU, and the polynomial's
-// extra issue slots on the MMA thread's sub-partition slow it (by 5-8% at 3 of
-// 8 pairs).
-constexpr int kPolyPairsPer8 = 0;
-__host__ __device__ constexpr bool poly_column_pair(int pair) { return (pair & 7) < kPolyPairsPer8; }
-
 __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
@@ -160,36 +137,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, got);
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
-// Rotate query row `row` (position i) of the Q tiles in shared memory (two
-// 64-dim boxes, 128-byte swizzle): pairs (k, k + r/2) for k < r/2.  Vector
-// form for 16 | r.  Both head slots' tiles hold the same query rows, so the
-// slots split a row's 8-pair chunks between them (slot s takes chunks
-// c0 = s, s+2, s+4, s+6) and each rotates its chunks in both tiles: every
-// table slice crosses from L2 once per work tile.  tb holds the thread's
-// 16-byte slices (two pairs each), loaded before the tiles' arrival is
-// awaited; the warp's 32 rows load each slice index from 512 contiguous
-// bytes.
-__device__ __forceinline__ void rope_table_load(float4 (&tb)[16], const float4* __restrict__ tgroup, int half,
-                                                int slot) {
-  // slices past half/2 repeat the last one: unconditional loads stay in registers
-  const int last = half / 2 - 1;
-#pragma unroll
-  for (int ci = 0; ci < 4; ++ci)
-#pragma unroll
-    for (int w = 0; w < 4; ++w) tb[4 * ci + w] = __ldg(tgroup + (size_t)min((2 * ci + slot) * 4 + w, last) * 32);
-}
-
-// Rotates dims 8 c0 .. 8 c0 + 7 with their partners 8 c0 + half .. of one row;
-// t4[w] holds (cos, sin) of pairs 8 c0 + 2w and 8 c0 + 2w + 1.
+// Rotates dims 8 c0 .. 8 c0 + 7 with their partners 8 c0 + half .. of one
+// row of a Q tile in shared memory (two 64-dim boxes, 128-byte swizzle);
+// t4[w] holds (cos, sin) of pairs 8 c0 + 2w and 8 c0 + 2w + 1.  Rounding as
+// in the RoPE kernels (the partner's product rounded, then one fma), so a
+// rotated q equals swa_rope_qk's bit for bit.
 __device__ __forceinline__ void rotate_q_chunk(uint8_t* tile, int row, int c0, int half, const float4* t4) {
   const int ea = c0 * 8, eb = ea + half;
   uint4* pa = reinterpret_cast<uint4*>(tile + (ea >> 6) * kBoxBytes + sw128_off(row, (ea & 63) >> 3));
@@ -202,25 +154,11 @@ __device__ __forceinline__ void rotate_q_chunk(uint8_t* tile, int row, int c0, i
     const float4 t = t4[w];
     const float x0 = bf16_lo(a32[w]), x1 = bf16_hi(a32[w]);
     const float y0 = bf16_lo(b32[w]), y1 = bf16_hi(b32[w]);
-    // the partner's product rounded, then one fma: the RoPE kernels' form,
-    // so a rotated q equals swa_rope_qk's bit for bit
     a32[w] = pack_bf16x2(fmaf(x0, t.x, -(y0 * t.y)), fmaf(x1, t.z, -(y1 * t.w)));
     b32[w] = pack_bf16x2(fmaf(y0, t.x, x0 * t.y), fmaf(y1, t.z, x1 * t.w));
   }
   *pa = A;
   *pb = Bv;
-}
-
-__device__ __forceinline__ void rotate_q_rows_vec(uint8_t* q0, uint8_t* q1, int row, int half, int slot,
-                                                  const float4 (&tb)[16]) {
-#pragma unroll
-  for (int ci = 0; ci < 4; ++ci) {
-    const int c0 = 2 * ci + slot;
-    if (c0 * 8 < half) {
-      rotate_q_chunk(q0, row, c0, half, tb + 4 * ci);
-      rotate_q_chunk(q1, row, c0, half, tb + 4 * ci);
-    }
-  }
 }
 
 // Element-wise form for any even r.
@@ -244,8 +182,7 @@ __device__ __forceinline__ void rotate_q_row_scalar(uint8_t* tile, int row, int 
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap q_map,
-                   const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
-                   const __grid_constant__ CUtensorMap o_map) {
+                   const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need 1024-byte alignment and the layout has
   // no room to realign: leave (uniformly, before any barrier) if it is off
@@ -253,34 +190,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) record_error(kErrPrefill + 15);
     return;
   }
-  PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>(smem_raw);
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = a.n_q_tiles * a.n_head_pairs * a.Hkv * a.B;
 
   if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(&sm.q_full[b][s], 1);
+        mbar_init(&sm.q_empty[b][s], 1);
+        mbar_init(&sm.l_full[b][s], BM);
+      }
+      mbar_init(&sm.q_ready[b], BM);
+    }
+    for (int i = 0; i < kKvStages; ++i) {
+      mbar_init(&sm.kv_full[i], 1);
+      mbar_init(&sm.kv_empty[i], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.q_full[s], 1);
-      mbar_init(&sm.q_empty[s], 1);
-      mbar_init(&sm.alpha_full[s], BM);
-      mbar_init(&sm.alpha_empty[s], BM);
-      mbar_init(&sm.l_full[s], BM);
-      mbar_init(&sm.l_empty[s], BM);
-      mbar_init(&sm.ost_full[s], BM);
-      mbar_init(&sm.pfree[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], BM);
+      mbar_init(&sm.o_done[s], 1);
+      mbar_init(&sm.o_free[s], BM);
     }
-    for (int i = 0; i < NK; ++i) {
-      mbar_init(&sm.k_full[i], 1);
-      mbar_init(&sm.k_empty[i], 1);
-    }
-    for (int i = 0; i < NV; ++i) {
-      mbar_init(&sm.v_full[i], 1);
-      mbar_init(&sm.v_empty[i], 1);
-    }
-    mbar_init(&sm.q_ready, 2 * BM);
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.pv_done, 1);
-    mbar_init(&sm.s_free, 2 * BM + 1);
-    mbar_init(&sm.pv_ready, 4 * BM + 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -298,287 +230,196 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 12) {
     regs_decrease<kRegsOther>();
     if (warp == 13 && lane == 0) {
-      // ========================================================== producer
-      // Per work tile: K(0), then [K(j+1), V(j)] per key tile (K runs one
-      // ahead, its 2-deep ring frees early; V's single buffer frees when both
-      // slots' P.V of the previous key tile complete).  The next tile's Q is
-      // loaded as soon as this tile's last QK^T has read Q.  No L2 prefetches
-      // (of the next V, or of a later tile's Q and cos/sin rows): with them
-      // the loads queued behind land later and the step is about 2 % slower.
-      prefetch_tensormap(&q_map);
+      // ========================================================== K / V producer
+      // Every key tile j of every work tile, in the order the MMAs consume
+      // them: K(j), V(j), into a three-stage ring.
       prefetch_tensormap(&k_map);
       prefetch_tensormap(&v_map);
-      int it = 0, kc = 0, vc = 0;           // tile counter, K / V loads issued
-      int k_end = 0, v_end = 0;             // loads issued (for the abort drain)
-      int q_last[2] = {-1, -1};
+      int idx = 0;
       bool ok = true;
-      auto load_q = [&](int t_q, int it_q) -> bool {
-        const Tile N = decode_tile<kMode>(a, t_q);
-        for (int s = 0; s < 2; ++s) {
-          if (it_q > 0 && !mbar_wait(&sm.q_empty[s], (it_q - 1) & 1, abort_flag)) return false;
-          mbar_arrive_expect_tx(&sm.q_full[s], kTileBytes);
-          const int h = s ? N.h1 : N.h0;
-          tma_load_4d(sm.q[s], &q_map, &sm.q_full[s], 0, h, N.r0, N.b);
-          tma_load_4d(sm.q[s] + kBoxBytes, &q_map, &sm.q_full[s], 64, h, N.r0, N.b);
-          q_last[s] = it_q;
-        }
-        return true;
-      };
-      auto load_kv = [&](bool is_v, const Tile& T, int j) -> bool {
-        const int idx = is_v ? vc++ : kc++;
-        const int nb = is_v ? NV : NK;
-        const int buf = idx % nb, use = idx / nb;
-        uint64_t* full = is_v ? &sm.v_full[buf] : &sm.k_full[buf];
-        uint64_t* empty = is_v ? &sm.v_empty[buf] : &sm.k_empty[buf];
-        if (use > 0 && !mbar_wait(empty, (use - 1) & 1, abort_flag)) return false;
-        uint8_t* dst = is_v ? sm.v[buf] : sm.k[buf];
-        const CUtensorMap* map = is_v ? &v_map : &k_map;
-        const int key0 = (T.kt_lo + j) * BN;
-        mbar_arrive_expect_tx(full, kTileBytes);
-        if constexpr (kMode == kChunkCache) {  // KV cache [B * Hkv, C, D]
-          tma_load_3d(dst, map, full, 0, key0, T.b * a.Hkv + T.kvh);
-          tma_load_3d(dst + kBoxBytes, map, full, 64, key0, T.b * a.Hkv + T.kvh);
-        } else {
-          tma_load_4d(dst, map, full, 0, T.kvh, key0, T.b);
-          tma_load_4d(dst + kBoxBytes, map, full, 64, T.kvh, key0, T.b);
-        }
-        if (is_v)
-          v_end = idx + 1;
-        else
-          k_end = idx + 1;
-        return true;
-      };
-      if (blockIdx.x < (unsigned)n_tiles && !load_q(blockIdx.x, 0)) ok = false;
-      for (int t = blockIdx.x; t < n_tiles && ok && !*abort_flag; t += gridDim.x, ++it) {
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         const Tile T = decode_tile<kMode>(a, t);
-        const bool has_next = t + (int)gridDim.x < n_tiles;
-        for (int j = -1; j < T.n_kv && ok; ++j) {
-          if (j + 1 < T.n_kv) ok = load_kv(false, T, j + 1);
-          if (ok && j >= 0) {
-            // the next tile's Q waits for this tile's last QK^T: issue it
-            // before the last V (which waits for the previous P.V), or after
-            // the only V of a one-key-tile tile
-            const bool last = j == T.n_kv - 1;
-            if (last && has_next && T.n_kv >= 2) ok = load_q(t + gridDim.x, it + 1);
-            if (ok) ok = load_kv(true, T, j);
-            if (ok && last && has_next && T.n_kv == 1) ok = load_q(t + gridDim.x, it + 1);
+        for (int j = 0; j < T.n_kv && ok; ++j) {
+          const int key0 = (T.kt_lo + j) * BN;
+          for (int v = 0; v < 2; ++v, ++idx) {
+            const int st = idx % kKvStages;
+            if (idx >= kKvStages && !mbar_wait(&sm.kv_empty[st], (idx / kKvStages - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const CUtensorMap* map = v ? &v_map : &k_map;
+            uint8_t* dst = sm.kv[st];
+            mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
+            if constexpr (kMode == kChunkCache) {  // KV cache [B * Hkv, C, D]
+              tma_load_3d(dst, map, &sm.kv_full[st], 0, key0, T.b * a.Hkv + T.kvh);
+              tma_load_3d(dst + kBoxBytes, map, &sm.kv_full[st], 64, key0, T.b * a.Hkv + T.kvh);
+            } else {
+              tma_load_4d(dst, map, &sm.kv_full[st], 0, T.kvh, key0, T.b);
+              tma_load_4d(dst + kBoxBytes, map, &sm.kv_full[st], 64, T.kvh, key0, T.b);
+            }
           }
         }
-        if (!ok) fail(abort_flag, kErrPrefill + 1);
       }
-      if (*abort_flag) {
+      if (!ok) {
+        fail(abort_flag, kErrPrefill + 1);
         // let every copy this thread started land before the CTA exits
-        for (int s = 0; s < 2; ++s)
-          if (q_last[s] >= 0) mbar_wait(&sm.q_full[s], q_last[s] & 1, nullptr, 200000000ull);
-        for (int g = k_end > NK ? k_end - NK : 0; g < k_end; ++g)
-          mbar_wait(&sm.k_full[g % NK], (g / NK) & 1, nullptr, 200000000ull);
-        for (int g = v_end > NV ? v_end - NV : 0; g < v_end; ++g)
-          mbar_wait(&sm.v_full[g % NV], (g / NV) & 1, nullptr, 200000000ull);
+        for (int g = idx > kKvStages ? idx - kKvStages : 0; g < idx; ++g)
+          mbar_wait(&sm.kv_full[g % kKvStages], (g / kKvStages) & 1, nullptr, 200000000ull);
+      }
+    } else if (warp == 15 && lane == 0) {
+      // ========================================================== Q producer
+      // Q of tile it goes to buffer it & 1 once the last QK^T of tile it - 2
+      // (the buffer's previous tile) has completed.
+      prefetch_tensormap(&q_map);
+      int it = 0, last_it = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+        const Tile N = decode_tile<kMode>(a, t);
+        const int b = it & 1;
+        for (int s = 0; s < 2; ++s) {
+          if (it >= 2 && !mbar_wait(&sm.q_empty[b][s], ((it - 2) >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int h = s ? N.h1 : N.h0;
+          mbar_arrive_expect_tx(&sm.q_full[b][s], kTileBytes);
+          tma_load_4d(sm.q[b][s], &q_map, &sm.q_full[b][s], 0, h, N.r0, N.b);
+          tma_load_4d(sm.q[b][s] + kBoxBytes, &q_map, &sm.q_full[b][s], 64, h, N.r0, N.b);
+        }
+        if (ok) last_it = it;
+      }
+      if (!ok) {
+        fail(abort_flag, kErrPrefill + 2);
+        for (int i = last_it > 0 ? last_it - 1 : 0; i <= last_it; ++i)
+          for (int s = 0; s < 2; ++s) mbar_wait(&sm.q_full[i & 1][s], (i >> 1) & 1, nullptr, 200000000ull);
       }
     } else if (warp == 12 && lane == 0) {
       // ========================================================== MMA issuer
-      // In-phase order per key tile: [S_0(j+1), S_1(j+1)] then [O_0 += P_0 V_j,
-      // O_1 += P_1 V_j], each pair issued one MMA of each GEMM in turn.  S(j+1)
-      // needs only that the softmax has read S(j) (P is in shared memory), so
-      // both QK^T of the next key tile overlap the softmax and the P.V of the
-      // current one: up to four independent accumulation chains in the pipe,
-      // where a lone chain of dependent tcgen05.mma runs at a fraction of its
-      // rate.  Descriptors advance by adding (byte offset >> 4) to the
-      // start-address field (no carry below 256 KB).
+      // Per key tile j and slot s: [O_s (+)= P_s(j) V(j); S_s = Q_s K(j+1)^T],
+      // where after a tile's last key tile K(j+1) is the next tile's first
+      // key tile and Q_s the next tile's buffer.  Ring index of K(j) in a tile
+      // is base + 2j, of V(j) base + 2j + 1.  Descriptors advance by adding
+      // (byte offset >> 4) to the start-address field in their low word.
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, 128, false, true);
-      const uint64_t qd0 = sw128_desc(smem_u32(sm.q[0]), 16, 1024), qd1 = sw128_desc(smem_u32(sm.q[1]), 16, 1024);
-      const uint64_t pd0 = sw128_desc(smem_u32(sm.p[0]), 16, 1024), pd1 = sw128_desc(smem_u32(sm.p[1]), 16, 1024);
-      const uint64_t kdesc0 = sw128_desc(smem_u32(sm.k[0]), 16, 1024);
-      const uint64_t vdesc0 = sw128_desc(smem_u32(sm.v[0]), kBoxBytes, 1024);
-      int it = 0, G = 0, kc = 0, vc = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const int n_kv = decode_tile<kMode>(a, t).n_kv;
-        if (!mbar_wait(&sm.q_ready, it & 1, abort_flag)) {
-          fail(abort_flag, kErrPrefill + 3);
-          ok = false;
-          break;
+      // the buffers are contiguous, so a buffer's descriptor is the first
+      // one's plus its byte offset >> 4 (no carry: shared memory < 256 KB)
+      const uint64_t qd = sw128_desc(smem_u32(sm.q[0][0]), 16, 1024);
+      const uint64_t kd = sw128_desc(smem_u32(sm.kv[0]), 16, 1024);
+      const uint64_t vd = sw128_desc(smem_u32(sm.kv[0]), kBoxBytes, 1024);
+      const uint32_t qlo = (uint32_t)qd, qhi = (uint32_t)(qd >> 32);
+      const uint32_t klo = (uint32_t)kd, khi = (uint32_t)(kd >> 32);
+      const uint32_t vlo = (uint32_t)vd, vhi = (uint32_t)(vd >> 32);
+      auto wait_kv = [&](int idx) -> bool {
+        return mbar_wait(&sm.kv_full[idx % kKvStages], (idx / kKvStages) & 1, abort_flag);
+      };
+      auto issue_qk = [&](int b, int s, int kidx) {
+        const uint32_t a0 = qlo + (uint32_t)(((b * 2 + s) * kTileBytes) >> 4);
+        const uint32_t b0 = klo + (uint32_t)(((kidx % kKvStages) * kTileBytes) >> 4), d = tmem + s * 128;
+#pragma unroll 2
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (uint32_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
+          umma_ss_lh(d, a0 + off, qhi, b0 + off, khi, idesc_qk, kk > 0);
         }
-        for (int j = -1; j < n_kv && ok; ++j) {
-          if (j + 1 < n_kv) {
-            const int g1 = G + j + 1, ki = kc + j + 1;
-            // s_free(g1 - 1) includes the arrival of K(g1); only the very
-            // first K tile is awaited here
-            ok = g1 == 0 ? mbar_wait(&sm.k_full[0], 0, abort_flag) : mbar_wait(&sm.s_free, (g1 - 1) & 1, abort_flag);
+      };
+      auto issue_pv = [&](int s, int vidx, bool acc) {
+        const uint32_t b0 = vlo + (uint32_t)(((vidx % kKvStages) * kTileBytes) >> 4);
+        const uint32_t d = tmem + 256 + s * 128, pa = tmem + s * 128;
+#pragma unroll 2
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts_lh(d, pa + kk * 8, b0 + (uint32_t)((kk * 2048) >> 4), vhi, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = true;
+      int it = 0, g = 0, base = 0;
+      if ((int)blockIdx.x < n_tiles) {
+        const Tile T0 = decode_tile<kMode>(a, blockIdx.x);
+        ok = mbar_wait(&sm.q_ready[0], 0, abort_flag) && wait_kv(0);
+        if (ok) {
+          tc_fence_after();
+          for (int s = 0; s < 2; ++s) {
+            issue_qk(0, s, 0);
+            umma_commit(&sm.s_full[s]);
+            if (T0.n_kv == 1) umma_commit(&sm.q_empty[0][s]);
+          }
+          umma_commit(&sm.kv_empty[0]);
+        } else {
+          fail(abort_flag, kErrPrefill + 3);
+        }
+      }
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+        const int n = decode_tile<kMode>(a, t).n_kv;
+        const bool has_next = t + (int)gridDim.x < n_tiles;
+        const int n_next = has_next ? decode_tile<kMode>(a, t + gridDim.x).n_kv : 0;
+        const int b = it & 1, nb = b ^ 1;
+        for (int j = 0; j < n && ok; ++j) {
+          const bool last = j == n - 1;
+          const int vidx = base + 2 * j + 1, kidx = base + 2 * j + 2;
+          for (int s = 0; s < 2 && ok; ++s) {
+            ok = mbar_wait(&sm.p_full[s], (g + j) & 1, abort_flag) &&
+                 (j > 0 || it == 0 || mbar_wait(&sm.o_free[s], (it - 1) & 1, abort_flag)) &&
+                 (s == 1 || wait_kv(vidx));
             if (!ok) {
               fail(abort_flag, kErrPrefill + 4);
               break;
             }
             tc_fence_after();
-            const uint64_t kd = kdesc0 + (uint64_t)(((ki % NK) * kTileBytes) >> 4);
-            // unrolled by 2, descriptors advanced in their low words: fewer
-            // instructions between MMAs on the issuer's busy sub-partition (C2
-            // -1.7 % and -2.2 %, C3 -2.9 % and -2.1 %; fully unrolled it spills at
-            // this warp's 56 registers, by 4 it ran slower)
-#pragma unroll 2
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t off = (uint64_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
-              const uint32_t o32 = (uint32_t)off;
-              umma_ss_lh(tmem, (uint32_t)qd0 + o32, (uint32_t)(qd0 >> 32), (uint32_t)kd + o32, (uint32_t)(kd >> 32),
-                         idesc_qk, kk > 0);
-              umma_ss_lh(tmem + 128, (uint32_t)qd1 + o32, (uint32_t)(qd1 >> 32), (uint32_t)kd + o32,
-                         (uint32_t)(kd >> 32), idesc_qk, kk > 0);
+            issue_pv(s, vidx, j > 0);
+            if (s == 1) umma_commit(&sm.kv_empty[vidx % kKvStages]);
+            if (last) umma_commit(&sm.o_done[s]);
+            if (!last || has_next) {
+              if (s == 0) {
+                ok = (!last || mbar_wait(&sm.q_ready[nb], ((it + 1) >> 1) & 1, abort_flag)) && wait_kv(kidx);
+                if (!ok) {
+                  fail(abort_flag, kErrPrefill + 5);
+                  break;
+                }
+                tc_fence_after();
+              }
+              issue_qk(last ? nb : b, s, kidx);
+              umma_commit(&sm.s_full[s]);
+              if (s == 1) umma_commit(&sm.kv_empty[kidx % kKvStages]);
+              // the last QK^T that reads this Q buffer frees it for a later tile
+              if (!last && j + 2 == n) umma_commit(&sm.q_empty[b][s]);
+              if (last && n_next == 1) umma_commit(&sm.q_empty[nb][s]);
             }
-            umma_commit(&sm.s_full);
-            umma_commit(&sm.k_empty[ki % NK]);
-            if (j + 2 == n_kv) {
-              umma_commit(&sm.q_empty[0]);
-              umma_commit(&sm.q_empty[1]);
-            }
-          }
-          if (j >= 0) {
-            const int g = G + j, vi = vc + j;
-            ok = mbar_wait(&sm.pv_ready, g & 1, abort_flag);  // includes the arrival of V(g)
-            if (!ok) {
-              fail(abort_flag, kErrPrefill + 5);
-              break;
-            }
-            tc_fence_after();
-            const uint64_t vd = vdesc0 + (uint64_t)(((vi % NV) * kTileBytes) >> 4);
-#pragma unroll 2
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t aoff = (uint64_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
-              const uint64_t boff = (uint64_t)((kk * 2048) >> 4);
-              const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-              umma_ss_lh(tmem + 256, (uint32_t)pd0 + (uint32_t)aoff, (uint32_t)(pd0 >> 32), (uint32_t)vd + (uint32_t)boff,
-                         (uint32_t)(vd >> 32), idesc_pv, acc);
-              umma_ss_lh(tmem + 384, (uint32_t)pd1 + (uint32_t)aoff, (uint32_t)(pd1 >> 32), (uint32_t)vd + (uint32_t)boff,
-                         (uint32_t)(vd >> 32), idesc_pv, acc);
-            }
-            umma_commit(&sm.pv_done);
-            umma_commit(&sm.v_empty[vi % NV]);
           }
         }
-        G += n_kv;
-        kc += n_kv;
-        vc += n_kv;
+        g += n;
+        base += 2 * n;
       }
       // all MMAs issued by this thread complete before the CTA moves on
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, nullptr, 200000000ull);
-    } else if (warp == 15 && lane == 0) {
-      // ========================================================== arrivals
-      // Folds the landing of each K / V tile into the barrier the MMA thread
-      // waits on anyway: s_free(g - 1) counts the arrival of K(g), pv_ready(g)
-      // that of V(g), in the issuer's order.  Before arriving for a phase it
-      // waits for the previous phase to complete, so an early arrival never
-      // counts toward the wrong phase.
-      int G = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int n_kv = decode_tile<kMode>(a, t).n_kv;
-        for (int j = -1; j < n_kv && ok; ++j) {
-          const int g1 = G + j + 1;
-          if (j + 1 < n_kv && g1 >= 1) {
-            ok = (g1 < 2 || mbar_wait(&sm.s_free, (g1 - 2) & 1, abort_flag)) &&
-                 mbar_wait(&sm.k_full[g1 % NK], (g1 / NK) & 1, abort_flag);
-            if (ok) mbar_arrive(&sm.s_free);
-          }
-          if (ok && j >= 0) {
-            const int g = G + j;
-            ok = (g < 1 || mbar_wait(&sm.pv_ready, (g - 1) & 1, abort_flag)) &&
-                 mbar_wait(&sm.v_full[g % NV], (g / NV) & 1, abort_flag);
-            if (ok) mbar_arrive(&sm.pv_ready);
-          }
-        }
-        G += n_kv;
-      }
-      if (!ok) fail(abort_flag, kErrPrefill + 18);
-    } else if (warp == 14 && lane == 0) {
-      // ========================================================== output store
-      // The epilogue stages each slot's output tile in that slot's P buffer;
-      // this thread stores it with TMA and frees the buffer once it is read.
-      prefetch_tensormap(&o_map);
-      int it = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-        const Tile T = decode_tile<kMode>(a, t);
-        bool ok = true;
-        for (int s = 0; s < 2; ++s) {
-          if (!mbar_wait(&sm.ost_full[s], it & 1, abort_flag)) {
-            fail(abort_flag, kErrPrefill + 14);
-            ok = false;
-            break;
-          }
-          if (s == 0 || T.store1) {
-            const int h = s ? T.h1 : T.h0;
-            tma_store_4d(&o_map, sm.p[s], 0, h, T.r0, T.b);
-            tma_store_4d(&o_map, sm.p[s] + kBoxBytes, 64, h, T.r0, T.b);
-            bulk_commit_group();
-          }
-          bulk_wait_group_read0();
-          mbar_arrive(&sm.pfree[s]);
-        }
-        if (!ok) break;
-      }
-      bulk_wait_group0();
     }
   } else if (warp < 8) {
     // ============================================================ softmax
     regs_increase<kRegsSoftmax>();
     const int s = warp >> 2;
     const int row = threadIdx.x & (BM - 1);
-    const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + s * 128;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + s * 128;
+    const uint32_t o_addr = tmem + lane_base + 256 + s * 128;
     const float c = a.scale_log2;
-    int it = 0, G = 0;
+    int it = 0, g = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile<kMode>(a, t);
-      const int r = T.r0 + row;  // query row
-      const int i = T.i0 + row;  // its key-space position
-      // ---- RoPE of the Q tiles (rows at or beyond S stay as loaded: zero);
-      // the table slices are requested before Q is awaited.  Vector form:
-      // this slot's half of each row's chunks in both tiles; scalar form:
-      // this slot's own tile.
-      {
-        const int half = a.rotary_dim / 2;
-        const bool rot = a.rotary_dim > 0 && r < a.S;
-        const bool vec = (half & 7) == 0;
-        const float4* tgroup = reinterpret_cast<const float4*>(a.table) +
-                               ((((size_t)(r >> 5) * rope_table_couples(half)) << 5) + (r & 31));
-        float4 tb[16];
-        if (rot && vec) {
-          rope_table_load(tb, tgroup, half, s);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) tb[k] = make_float4(1.f, 0.f, 1.f, 0.f);
-        }
-        if (!warp_wait(&sm.q_full[0], it & 1, abort_flag) || !warp_wait(&sm.q_full[1], it & 1, abort_flag)) {
-          fail(abort_flag, kErrPrefill + 6);
-          ok = false;
-          break;
-        }
-        if (rot) {
-          if (vec)
-            rotate_q_rows_vec(sm.q[0], sm.q[1], row, half, s, tb);
-          else
-            rotate_q_row_scalar(sm.q[s], row, r, half, a.table);
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&sm.q_ready);
-      }
+      const int i = T.i0 + row;  // key-space position of this row
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < T.n_kv; ++j) {
+      for (int j = 0; j < T.n_kv; ++j, ++g) {
         const int key0 = (T.kt_lo + j) * BN;
-        if (!warp_wait(&sm.s_full, (G + j) & 1, abort_flag)) {
+        if (!warp_wait(&sm.s_full[s], g & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 7);
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t v[128];
-        tmem_ld32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
-        tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
-        tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+        tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+        tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&sm.s_free);  // S_s may be overwritten by the next QK^T
         // which mask bounds cut this key tile (uniform over the tile):
         // hi -- some key lies after some row (the diagonal tile);
         // lo -- some key lies at or before row - W (the band's first tile).
@@ -589,8 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool cut_lo = a.window > 0 && key0 < T.i0 + BM - a.window;
         uint32_t masked = 0;  // bit q: chunk q masked for every row of the warp
         if (cut_hi || cut_lo) {
-          const int hi = cut_hi ? i - key0 : BN;                     // columns > hi are masked
-          const int lo = cut_lo ? i - a.window + 1 - key0 : -1;      // columns < lo are masked
+          const int hi = cut_hi ? i - key0 : BN;                 // columns > hi are masked
+          const int lo = cut_lo ? i - a.window + 1 - key0 : -1;  // columns < lo are masked
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int c0 = 32 * q;
@@ -616,15 +457,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_use = (mt - m > kRescaleThreshold) ? mt : m;  // m = -inf: always take mt
         const float m_safe = m_use == -INFINITY ? 0.f : m_use;
         const float alpha = fast_exp2(m - m_safe);
-        // the correction has read the previous alpha (the softmax can run a
-        // key tile ahead of it now that S(j+1) no longer waits for P(j).V)
-        if (G + j > 0 && !warp_wait(&sm.alpha_empty[s], (G + j - 1) & 1, abort_flag)) {
-          fail(abort_flag, kErrPrefill + 17);
-          ok = false;
-          break;
-        }
-        sm.alpha[s][row] = alpha;
-        mbar_arrive(&sm.alpha_full[s]);
         // P = 2^(c S - m), two columns per packed FMA; masked columns give 0
         const uint64_t cc = f2_pack(c, c), mm = f2_pack(-m_safe, -m_safe);
         uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
@@ -638,137 +470,150 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 32 * q; e < 32 * q + 32; e += 2) {
               const uint64_t y = f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), cc, mm);
-              float p0, p1;
-              if (poly_column_pair(e >> 1)) {
-                f2_unpack(exp2_poly2(y), p0, p1);
-              } else {
-                float y0, y1;
-                f2_unpack(y, y0, y1);
-                p0 = fast_exp2(y0);
-                p1 = fast_exp2(y1);
-              }
+              float y0, y1;
+              f2_unpack(y, y0, y1);
+              const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
               sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(p0, p1));
               pk[e >> 1] = pack_bf16x2(p0, p1);
             }
           }
         }
-        // p[s] is free once P_s(j-1).V has completed; at a tile's first key
-        // tile it holds the previous tile's output until the store has read
-        // it.  (S(j) completing implies P(j-2).V completed, since its commit
-        // covers every earlier MMA, so these waits are never two phases ahead.)
-        if (j > 0 ? !warp_wait(&sm.pv_done, (G + j - 1) & 1, abort_flag)
-                  : (it > 0 && !warp_wait(&sm.pfree[s], (it - 1) & 1, abort_flag))) {
-          fail(abort_flag, kErrPrefill + 16);
-          ok = false;
-          break;
-        }
+        // P over the S columns it came from (S is in registers already)
+        tmem_st32(s_addr + 0, *reinterpret_cast<const uint32_t(*)[32]>(pk + 0));
+        tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+        // O_s holds key tiles 0..j-1 (their P.V completed before S(j) did):
+        // bring it to the new max before P(j).V adds to it
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t o[32];
+            tmem_ld32(o_addr + q4 * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch)
-          *reinterpret_cast<uint4*>(sm.p[s] + (ch >> 3) * kBoxBytes + sw128_off(row, ch & 7)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive(&sm.pv_ready);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(o_addr + q4 * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[s]);
         float s0, s1;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
         l = l * alpha + (s0 + s1);
         m = m_use;
       }
       if (!ok) break;
-      if (it > 0 && !warp_wait(&sm.l_empty[s], (it - 1) & 1, abort_flag)) {
-        fail(abort_flag, kErrPrefill + 8);
-        break;
-      }
-      sm.lsum[s][row] = l;
-      mbar_arrive(&sm.l_full[s]);
-      G += T.n_kv;
+      // double-buffered by tile parity: the epilogue of tile it - 2 read this
+      // slot before tile it's first P.V could start
+      sm.lsum[it & 1][s][row] = l;
+      mbar_arrive(&sm.l_full[it & 1][s]);
     }
   } else {
-    // ============================================================ correction
+    // ============================================================ Q rotation + epilogue
     regs_decrease<kRegsCorrection>();
     const int row = threadIdx.x & (BM - 1);
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    int it = 0, G = 0;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int half = a.rotary_dim / 2;
+    const bool vec = (half & 7) == 0;
+    // RoPE of the Q tiles of work tile tq (iteration itq) in buffer itq & 1,
+    // both head slots, this thread's row (rows at or beyond S stay as
+    // loaded: zero)
+    auto rotate = [&](int tq, int itq) -> bool {
+      const Tile N = decode_tile<kMode>(a, tq);
+      const int b = itq & 1;
+      const int r = N.r0 + row;
+      const bool rot = half > 0 && r < a.S;
+      const float4* tgroup = reinterpret_cast<const float4*>(a.table) +
+                             ((((size_t)(r >> 5) * rope_table_couples(half)) << 5) + (r & 31));
+      // the next chunk's table slices (eight pairs) are in flight while the
+      // current chunk is applied; slices past the last chunk repeat it
+      const int n_chunks = half / 8;
+      float4 ta[4], tb[4];
+      auto load1 = [&](float4 (&t)[4], int c0) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) t[w] = __ldg(tgroup + (size_t)(4 * min(c0, n_chunks - 1) + w) * 32);
+      };
+      if (rot && vec) load1(ta, 0);
+      if (!warp_wait(&sm.q_full[b][0], (itq >> 1) & 1, abort_flag) ||
+          !warp_wait(&sm.q_full[b][1], (itq >> 1) & 1, abort_flag))
+        return false;
+      if (rot) {
+        if (vec) {
+          for (int c0 = 0; c0 < n_chunks; c0 += 2) {
+            load1(tb, c0 + 1);
+            rotate_q_chunk(sm.q[b][0], row, c0, half, ta);
+            rotate_q_chunk(sm.q[b][1], row, c0, half, ta);
+            if (c0 + 1 >= n_chunks) break;
+            load1(ta, c0 + 2);
+            rotate_q_chunk(sm.q[b][0], row, c0 + 1, half, tb);
+            rotate_q_chunk(sm.q[b][1], row, c0 + 1, half, tb);
+          }
+        } else {
+          rotate_q_row_scalar(sm.q[b][0], row, r, half, a.table);
+          rotate_q_row_scalar(sm.q[b][1], row, r, half, a.table);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.q_ready[b]);
+      return true;
+    };
+    int it = 0;
     bool ok = true;
+    if ((int)blockIdx.x < n_tiles && !rotate(blockIdx.x, 0)) {
+      fail(abort_flag, kErrPrefill + 6);
+      ok = false;
+    }
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
       const Tile T = decode_tile<kMode>(a, t);
       const int r = T.r0 + row;  // query row
       // gate logits of this row for both head slots, fetched early
-      float glog[2] = {0.f, 0.f};
+      float glog0 = 0.f, glog1 = 0.f;
       if (a.gate && r < a.S) {
-        glog[0] = __ldg(a.gate + ((size_t)T.b * a.S + r) * a.Hq + T.h0);
-        glog[1] = __ldg(a.gate + ((size_t)T.b * a.S + r) * a.Hq + T.h1);
+        glog0 = __ldg(a.gate + ((size_t)T.b * a.S + r) * a.Hq + T.h0);
+        glog1 = __ldg(a.gate + ((size_t)T.b * a.S + r) * a.Hq + T.h1);
       }
-      for (int j = 0; j < T.n_kv && ok; ++j) {
-        for (int s = 0; s < 2; ++s) {
-          if (!warp_wait(&sm.alpha_full[s], (G + j) & 1, abort_flag)) {
-            fail(abort_flag, kErrPrefill + 9);
-            ok = false;
-            break;
-          }
-          const float alpha = sm.alpha[s][row];
-          mbar_arrive(&sm.alpha_empty[s]);
-          if (j > 0) {
-            if (!warp_wait(&sm.pv_done, (G + j - 1) & 1, abort_flag)) {
-              fail(abort_flag, kErrPrefill + 10);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
-              const uint32_t oaddr = tmem + lane_off + 256 + s * 128;
-#pragma unroll 1
-              for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t v[32];
-                tmem_ld32(oaddr + q4 * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                tmem_st32(oaddr + q4 * 32, v);
-              }
-              tmem_wait_st();
-            }
-          }
-          tc_fence_before();
-          mbar_arrive(&sm.pv_ready);
-        }
+      if (t + (int)gridDim.x < n_tiles && !rotate(t + gridDim.x, it + 1)) {
+        fail(abort_flag, kErrPrefill + 8);
+        break;
       }
-      if (!ok) break;
-      // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged in p[s] for
-      // the store warp (P_s(last) is consumed once that slot's P.V is done)
+      // ---- epilogue: out = O / l * sigmoid(gate), bf16, straight to global
       for (int s = 0; s < 2 && ok; ++s) {
-        if (!warp_wait(&sm.pv_done, (G + T.n_kv - 1) & 1, abort_flag) ||
-            !warp_wait(&sm.l_full[s], it & 1, abort_flag)) {
+        if (!warp_wait(&sm.o_done[s], it & 1, abort_flag) ||
+            !warp_wait(&sm.l_full[it & 1][s], (it >> 1) & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 11);
           ok = false;
           break;
         }
         tc_fence_after();
-        const float l = sm.lsum[s][row];
-        mbar_arrive(&sm.l_empty[s]);
-        const float g = a.gate ? 1.f / (1.f + __expf(-glog[s])) : 1.f;
-        const float f = g / l;
-        uint8_t* stage = sm.p[s];
-        const uint32_t oaddr = tmem + lane_off + 256 + s * 128;
+        const float l = sm.lsum[it & 1][s][row];
+        const float gt = a.gate ? 1.f / (1.f + __expf(-(s ? glog1 : glog0))) : 1.f;
+        const float f = gt / l;
+        const bool store = r < a.S && (s == 0 || T.store1);
+        uint4* dst = reinterpret_cast<uint4*>(a.out + (((size_t)T.b * a.S + r) * a.Hq + (s ? T.h1 : T.h0)) * 128);
+        const uint32_t oaddr = tmem + lane_base + 256 + s * 128;
 #pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t v[32];
           tmem_ld32(oaddr + q4 * 32, v);
           tmem_wait_ld();
+          if (q4 == 3) {
+            // O_s is in registers: the next tile's first P.V may overwrite it
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[s]);
+          }
+          if (store) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int ch = q4 * 4 + c4;  // 16-byte chunk (8 dims) 0..15
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(v[8 * c4 + 0]) * f, __uint_as_float(v[8 * c4 + 1]) * f);
-            u.y = pack_bf16x2(__uint_as_float(v[8 * c4 + 2]) * f, __uint_as_float(v[8 * c4 + 3]) * f);
-            u.z = pack_bf16x2(__uint_as_float(v[8 * c4 + 4]) * f, __uint_as_float(v[8 * c4 + 5]) * f);
-            u.w = pack_bf16x2(__uint_as_float(v[8 * c4 + 6]) * f, __uint_as_float(v[8 * c4 + 7]) * f);
-            *reinterpret_cast<uint4*>(stage + (ch >> 3) * kBoxBytes + sw128_off(row, ch & 7)) = u;
+            for (int c4 = 0; c4 < 4; ++c4) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(v[8 * c4 + 0]) * f, __uint_as_float(v[8 * c4 + 1]) * f);
+              u.y = pack_bf16x2(__uint_as_float(v[8 * c4 + 2]) * f, __uint_as_float(v[8 * c4 + 3]) * f);
+              u.z = pack_bf16x2(__uint_as_float(v[8 * c4 + 4]) * f, __uint_as_float(v[8 * c4 + 5]) * f);
+              u.w = pack_bf16x2(__uint_as_float(v[8 * c4 + 6]) * f, __uint_as_float(v[8 * c4 + 7]) * f);
+              dst[q4 * 4 + c4] = u;
+            }
           }
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&sm.ost_full[s]);
       }
-      G += T.n_kv;
     }
   }
 
@@ -780,17 +625,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-}  // namespace prefill_detail
-
-namespace prefill_detail {
-
 template <int kMode>
 cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                             const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream) {
+                             const CUtensorMap& v_map, cudaStream_t stream) {
   const long long n_tiles = (long long)a.n_q_tiles * a.n_head_pairs * a.Hkv * a.B;
   if (n_tiles == 0) return cudaSuccess;
   if (n_tiles > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  const size_t smem = sizeof(PrefillSmem);
+  const size_t smem = sizeof(Smem);
   static DeviceOnce setup;
   int n_sm = 0;
   cudaError_t e = device_once(setup, [&](int dev, int* sm_count) -> cudaError_t {
@@ -807,18 +648,18 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& q_map, con
   }, &n_sm);
   if (e != cudaSuccess) return e;
   const int grid = (int)(n_tiles < n_sm ? n_tiles : n_sm);
-  return launch_kernel(false, prefill_kernel<kMode>, dim3(grid), dim3(kThreads), smem, stream, a, q_map, k_map, v_map,
-                          o_map);
+  return launch_kernel(false, prefill_kernel<kMode>, dim3(grid), dim3(kThreads), smem, stream, a, q_map, k_map,
+                       v_map);
 }
 
 }  // namespace prefill_detail
 
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                           const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream) {
+                            const CUtensorMap& v_map, cudaStream_t stream) {
   using namespace prefill_detail;
-  if (a.kv_cache_layout) return launch_prefill_t<kChunkCache>(a, q_map, k_map, v_map, o_map, stream);
-  if (a.q_off) return launch_prefill_t<kChunkSeq>(a, q_map, k_map, v_map, o_map, stream);
-  return launch_prefill_t<kWhole>(a, q_map, k_map, v_map, o_map, stream);
+  if (a.kv_cache_layout) return launch_prefill_t<kChunkCache>(a, q_map, k_map, v_map, stream);
+  if (a.q_off) return launch_prefill_t<kChunkSeq>(a, q_map, k_map, v_map, stream);
+  return launch_prefill_t<kWhole>(a, q_map, k_map, v_map, stream);
 }
 
 }  // namespace swa

@@ -194,6 +194,20 @@ __device__ __forceinline__ void umma_ss_lh(uint32_t d_tmem, uint32_t a_lo, uint3
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16: A (M rows on the lanes, two
+// bf16 per 32-bit column) is read from tensor memory, B from shared memory
+// (descriptor passed as its 32-bit halves, as in umma_ss_lh).
+__device__ __forceinline__ void umma_ts_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on an mbarrier when all tcgen05.mma issued so far by this
 // thread have completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -323,8 +337,8 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 // softmax otherwise saturates).  y is clamped to >= -127 and split as
 // y = n + f, n = round(y) via the 1.5 * 2^23 rounding constant, f in
 // [-1/2, 1/2]; 2^f comes from a cubic with constant term exactly 1 (minimax
-// relative error 1.01e-4 on the interval, fitted by exp2_poly_fit.py beside
-// this file) and n is added into the exponent field.  Inputs at or below
+// relative error 1.01e-4 on the interval, fitted by tests/exp2_poly_fit.py)
+// and n is added into the exponent field.  Inputs at or below
 // -127, -inf included, give +0.0 exactly: n = -127, f = 0, and the sum of the
 // bit patterns of 1.0 and -127 << 23 wraps to zero.  For y in [-126, 127] the
 // result is within that relative error of 2^y; between -127 and -126 it is a
