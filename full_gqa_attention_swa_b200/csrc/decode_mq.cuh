@@ -1,181 +1,119 @@
-// Multi-query decode: T new tokens of every sequence attend in one call, each
-// through its own band.  The "Step-3.7-Flash" spec card's architecture notes
-// list three extra multi-token-prediction (MTP) layers that speed up decoding;
-// the tokens they propose are checked this way.  The band and the cache rule
-// are the "Step-3.7-Flash-oQ3e" explainer's
+// Multi-query decode on the tensor cores: T new tokens of every sequence
+// attend in one call, each through its own band.  The "Step-3.7-Flash" spec
+// card's architecture notes list three extra multi-token-prediction (MTP)
+// layers that speed up decoding; the tokens they propose are checked this
+// way.  The band and the cache rule are the "Step-3.7-Flash-oQ3e" explainer's
 // section 2.2 (a sliding layer keeps the last W tokens; query i sees keys
 // i - W < j <= i), the gate its section 2.3.
 //
-// The cache holds the L0 = L - T earlier tokens (ring slot p mod W, or slot p);
-// the new tokens' rotated keys and values come separately, so checking drafts
-// never overwrites ring slots an earlier query still needs.  Query t sits at
-// position L0 + t.  On a ring, dist(s) = (s - n - 1) mod W numbers the slots
-// from the oldest (n = slot of position L0 - 1); query t loses exactly the
-// slots with dist <= t, and sees new key j iff t - W < j <= t.
+// The cache holds the L0 = L - T earlier tokens (ring slot p mod W, or slot
+// p); the new tokens' rotated keys and values come separately, so checking
+// drafts never overwrites ring slots an earlier query still needs.  Query t
+// sits at position L0 + t.  On a ring, dist(s) = (s - n - 1) mod W numbers the
+// slots from the oldest (n = slot of position L0 - 1); query t sees exactly the
+// slots with dist > t, and new key j iff t - W < j <= t.
 //
-// Work split: one CTA per (sequence, kv-head, split of the cache), as in the
-// one-query decode, but the M dimension of the m16n8k16 MMAs is now the
-// T * G (query, head) rows of the kv-head: warp w owns rows 16w .. 16w + 15
-// over every key of the split, so the warps never merge.  One elected thread
-// streams 32-key K/V stages with TMA (no producer warp: at 49 KB of stages and
-// at most 168 registers, four CTAs share an SM, so the 512 (sequence,
-// kv-head) pairs of a 64-sequence batch run in one wave); the last split also
-// runs one 16-key block of new tokens, staged into a free stage after the loop.
-// Cache bytes are still read once per (sequence, kv-head); the T-fold rows
-// raise the tensor work per byte, which stays far below the MMA rate.
+// Work split: one CTA per (sequence, kv-head, split of the cache).  The T * G
+// (query, head) rows of the kv-head (<= 64) are the M dimension of
+// tcgen05.mma (M = 128, rows past T * G are zero), so a key block costs the
+// tensor core a handful of instructions: S = Q K^T (N = 64 keys) into tensor
+// memory, the softmax (thread = row) writes P (bf16) over S, and
+// O += P V reads P from tensor memory.  S is double-buffered (two 64-column
+// tiles), so the QK^T of block j + 1 overlaps the softmax of block j.  K and V
+// stream through separate TMA rings (three and two 64-key stages).  At 96 KB
+// of shared memory and 256 tensor-memory columns a CTA, two CTAs share an SM.
+// The last split also runs one 16-key block of the new tokens.
 #pragma once
-#include "decode.cuh"
+#include "swa_internal.cuh"
 
 namespace swa {
 
 namespace decode_mq_detail {
 
-using decode_detail::KB;
-using decode_detail::kBoxBytes;
-using decode_detail::kStageBytes;
-using decode_detail::ldsm_x4;
-using decode_detail::ldsm_x4_t;
-using decode_detail::mma_bf16;
-using decode_detail::sigmoidf_;
-using decode_detail::sw128_off;
-
-constexpr int kNewRows = 16;  // new-token block (T <= 16), zero-padded, staged in stage 0
-constexpr int kStages = 3;
-// resident CTAs per SM: four (49 KB of shared memory each); four m-tiles
-// would spill at the register share of four, so they run three per SM
-constexpr int ctas_per_sm(int mt) { return mt <= 3 ? 4 : 3; }
+constexpr int KB = 64;                           // keys per cache block
+constexpr int kNewRows = 16;                     // new-token block (T <= 16)
+constexpr int kKStages = 3, kVStages = 2;
+constexpr uint32_t kBoxBytes = KB * 128;         // 64 rows x 64 bf16
+constexpr uint32_t kBlockBytes = 2 * kBoxBytes;  // 64 keys x 128 dims
+constexpr uint32_t kNewBoxBytes = kNewRows * 128;
+constexpr int kThreads = 160;                    // softmax warps 0-1, K producer 2, issuer 3, V producer 4
+constexpr uint32_t kTmemCols = 256;              // S0 [0,64) S1 [64,128) O [128,256)
 static_assert(kNewRows == kDecodeMqMaxT, "one block holds every new token");
-static_assert(ctas_per_sm(3) == decode_mq_ctas_per_sm(48) && ctas_per_sm(4) == decode_mq_ctas_per_sm(64),
-              "the split plan sees the kernel's occupancy");
-static_assert(kStageBytes % 1024 == 0 && kNewRows <= KB, "stage boxes stay 1024-byte aligned and hold the new rows");
+static_assert(kDecodeMqMaxRows <= 64, "rows fit the two softmax warps");
 
-struct MqSmem {
-  uint8_t stage[kStages][kStageBytes];  // K lo, K hi, V lo, V hi boxes of 32 keys
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+struct Smem {
+  uint8_t q[2 * kBoxBytes];                  // rows (t, g) < 64 of both 64-dim halves
+  uint8_t k[kKStages][kBlockBytes];
+  uint8_t v[kVStages][kBlockBytes];
+  uint64_t q_full;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
   int abort_flag;
 };
 
-// One warp's 16 rows: Q fragments, output accumulators, running max (log2
-// units) and per-lane partial sums of rows g and g + 8.
-struct RowState {
-  uint32_t qf[8][4];
-  float o[16][4];
-  float m0, m1, l0, l1;
-};
-
-// One block of NK keys: S = Q K^T, masked online softmax, O += P V.  The K/V
-// halves lie `box` bytes apart.  vis(kidx, hi) tells whether key kidx of the
-// block is visible to row g (hi = 0) or g + 8 (hi = 1).  Keys at or past
-// `live`, and key `dead` (a slot outside every query's band, or -1), are
-// never visible; their V rows are zeroed in registers, as they may hold NaN
-// and 0 * NaN would reach the sum.
-template <int NK, bool kMasked, class Vis>
-__device__ __forceinline__ void mq_block(RowState& R, uint32_t kbase, uint32_t vbase, uint32_t box, float c,
-                                         int lane, int live, int dead, Vis vis) {
-  constexpr int NT = NK / 8;
-  const int tig = lane & 3;
-  // S: the NT accumulation chains advance together, one 32-dim step at a
-  // time, so NT independent MMAs are in flight behind each other
-  float sc[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < 8; kk += 2) {
-    const int ch = 2 * kk + (lane >> 3);  // 16-byte chunk (8 dims) 0..15
-    uint32_t kb[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      ldsm_x4(kbase + (ch >> 3) * box + sw128_off(nt * 8 + (lane & 7), ch & 7), kb[nt][0], kb[nt][1], kb[nt][2],
-              kb[nt][3]);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], R.qf[kk], kb[nt][0], kb[nt][1]);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], R.qf[kk + 1], kb[nt][2], kb[nt][3]);
-  }
-  float p[NT][4];
-  float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float v = sc[nt][e] * c;
-      p[nt][e] = (!kMasked || vis(nt * 8 + 2 * tig + (e & 1), e >> 1)) ? v : -INFINITY;
-    }
-    mx0 = fmaxf(mx0, fmaxf(p[nt][0], p[nt][1]));
-    mx1 = fmaxf(mx1, fmaxf(p[nt][2], p[nt][3]));
-  }
-  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-  const float mn0 = fmaxf(R.m0, mx0), mn1 = fmaxf(R.m1, mx1);
-  const float ms0 = mn0 == -INFINITY ? 0.f : mn0, ms1 = mn1 == -INFINITY ? 0.f : mn1;
-  const float al0 = fast_exp2(R.m0 - ms0), al1 = fast_exp2(R.m1 - ms1);
-  R.m0 = mn0;
-  R.m1 = mn1;
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    p[nt][0] = fast_exp2(p[nt][0] - ms0);
-    p[nt][1] = fast_exp2(p[nt][1] - ms0);
-    p[nt][2] = fast_exp2(p[nt][2] - ms1);
-    p[nt][3] = fast_exp2(p[nt][3] - ms1);
-    s0 += p[nt][0] + p[nt][1];
-    s1 += p[nt][2] + p[nt][3];
-  }
-  R.l0 = R.l0 * al0 + s0;
-  R.l1 = R.l1 * al1 + s1;
-#pragma unroll
-  for (int n = 0; n < 16; ++n) {
-    R.o[n][0] *= al0; R.o[n][1] *= al0;
-    R.o[n][2] *= al1; R.o[n][3] *= al1;
-  }
-  const int mi = lane >> 3;
-#pragma unroll
-  for (int ks = 0; ks < NK / 16; ++ks) {
-    uint32_t pa[4];
-    pa[0] = pack_bf16x2(p[2 * ks][0], p[2 * ks][1]);
-    pa[1] = pack_bf16x2(p[2 * ks][2], p[2 * ks][3]);
-    pa[2] = pack_bf16x2(p[2 * ks + 1][0], p[2 * ks + 1][1]);
-    pa[3] = pack_bf16x2(p[2 * ks + 1][2], p[2 * ks + 1][3]);
-    // this lane's B fragments hold keys k0, k0 + 1 (b0, b2) and k0 + 8, k0 + 9 (b1, b3)
-    const int k0 = ks * 16 + 2 * tig;
-    auto keep = [&](int k) -> bool { return k < live && k != dead; };
-    const uint32_t keep_lo = (keep(k0) ? 0x0000FFFFu : 0u) | (keep(k0 + 1) ? 0xFFFF0000u : 0u);
-    const uint32_t keep_hi = (keep(k0 + 8) ? 0x0000FFFFu : 0u) | (keep(k0 + 9) ? 0xFFFF0000u : 0u);
-    const bool sanitize = live < NK || (unsigned)dead < (unsigned)NK;
-    const int vrow = ks * 16 + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-    for (int n = 0; n < 16; n += 2) {
-      const int ch = n + (mi >> 1);  // dims 8*ch .. 8*ch+7
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(vbase + (ch >> 3) * box + sw128_off(vrow, ch & 7), b0, b1, b2, b3);
-      if (sanitize) {
-        b0 &= keep_lo; b2 &= keep_lo;
-        b1 &= keep_hi; b3 &= keep_hi;
-      }
-      mma_bf16(R.o[n], pa, b0, b1);
-      mma_bf16(R.o[n + 1], pa, b2, b3);
+// Wait that sleeps between tests, for roles whose waits are not on the
+// critical path (the TMA producers): a tight polling loop takes issue slots
+// from the softmax warps that share its sub-partition.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(ns);
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) return false;
     }
   }
 }
 
-// grid (max_splits, Hkv, B); MT warps of 16 rows each.  Lane 0 of warp 0
-// also issues the TMA loads: the first kStages blocks up front, then at the
-// top of step t the block t - 1 + kStages into the stage every warp released
-// after step t - 1.
-template <int MT>
-__global__ void __launch_bounds__(MT * 32, ctas_per_sm(MT))
-    decode_mq_kernel(const DecodeMqArgs a, const __grid_constant__ CUtensorMap k_map,
-                     const __grid_constant__ CUtensorMap v_map) {
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ float sigmoidf_(float g) { return 1.f / (1.f + __expf(-g)); }
+
+__device__ __forceinline__ void fail(volatile int* abort_flag, int code) {
+  record_error(code);
+  *abort_flag = 1;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool got = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, got);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// grid (max_splits, Hkv, B)
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_mq_kernel(const DecodeMqArgs a, const __grid_constant__ CUtensorMap q_map,
+                     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
+                     const __grid_constant__ CUtensorMap kn_map, const __grid_constant__ CUtensorMap vn_map) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  MqSmem& sm = *reinterpret_cast<MqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   allow_dependent_launch();
   grid_dependency_wait();
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int T = a.T;
+  const int T = a.T, G = a.G, n_rows = T * G;
   const int L0 = a.seq_lens[b] - T;  // cached tokens before the new ones
   const bool ring = a.window > 0;
   if (L0 < 0 || (!ring && L0 > a.capacity)) {  // uniform over the CTA, before any barrier
@@ -187,178 +125,341 @@ __global__ void __launch_bounds__(MT * 32, ctas_per_sm(MT))
   if (split >= n_split) return;
   const int k_begin = split * a.chunk;
   const int k_end = min(n_cache, k_begin + a.chunk);
-  const int n_blocks = k_end > k_begin ? (k_end - k_begin + KB - 1) / KB : 0;
+  const int n_cb = k_end > k_begin ? (k_end - k_begin + KB - 1) / KB : 0;  // cache blocks
   const bool has_new = split == n_split - 1;
+  const int n_tot = n_cb + (has_new ? 1 : 0);  // >= 1
   const int newest = (ring && L0 > 0) ? (L0 - 1) % a.window : 0;  // ring slot of position L0 - 1
-  // a full ring's oldest slot (position L0 - W) lies outside every query's band
-  const int dead_slot = (ring && L0 >= a.window) ? (newest + 1) % a.window : -1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool issuer = threadIdx.x == 0;
-  const int row3 = b * a.Hkv + kvh;
-  auto issue = [&](int t) {
-    const int s = t % kStages;
-    const int key0 = k_begin + t * KB;
-    uint8_t* st = sm.stage[s];
-    mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
-    tma_load_3d(st, &k_map, &sm.full[s], 0, key0, row3);
-    tma_load_3d(st + kBoxBytes, &k_map, &sm.full[s], 64, key0, row3);
-    tma_load_3d(st + 2 * kBoxBytes, &v_map, &sm.full[s], 0, key0, row3);
-    tma_load_3d(st + 3 * kBoxBytes, &v_map, &sm.full[s], 64, key0, row3);
-  };
-  int issued = 0;
-  if (issuer) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], MT);
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
     }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], 2);  // one arrival per softmax warp
+      mbar_init(&sm.pv_done[s], 1);
+    }
+    mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
-    if (n_blocks > 0) {
-      prefetch_tensormap(&k_map);
-      prefetch_tensormap(&v_map);
-    }
-    for (; issued < n_blocks && issued < kStages; ++issued) issue(issued);
   }
+  // rows n_rows .. 63 of Q stay zero (the TMA box writes only the first n_rows)
+  for (int i = threadIdx.x; i < (int)(2 * kBoxBytes / 16); i += kThreads)
+    reinterpret_cast<uint4*>(sm.q)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
+  const int row3 = b * a.Hkv + kvh;
 
-  const int g = lane >> 2, tig = lane & 3;
-  const int G = a.G, n_rows = T * G;
-  const int r0 = warp * 16 + g, r1 = r0 + 8;
-  const bool v0 = r0 < n_rows, v1 = r1 < n_rows;
-  const int t0 = v0 ? r0 / G : 0, t1 = v1 ? r1 / G : 0;
-  const int h0 = kvh * G + (v0 ? r0 % G : 0), h1 = kvh * G + (v1 ? r1 % G : 0);
-  const size_t row0 = ((size_t)b * T + t0) * a.Hq + h0, row1 = ((size_t)b * T + t1) * a.Hq + h1;
-
-  RowState R;
-  {
-    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + row0 * kHeadDim);
-    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + row1 * kHeadDim);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const int w0 = kk * 8 + tig;  // 32-bit word of dims (16kk + 2tig, +1)
-      R.qf[kk][0] = v0 ? __ldg(q0 + w0) : 0u;
-      R.qf[kk][1] = v1 ? __ldg(q1 + w0) : 0u;
-      R.qf[kk][2] = v0 ? __ldg(q0 + w0 + 4) : 0u;
-      R.qf[kk][3] = v1 ? __ldg(q1 + w0 + 4) : 0u;
-    }
-  }
-#pragma unroll
-  for (int n = 0; n < 16; ++n) R.o[n][0] = R.o[n][1] = R.o[n][2] = R.o[n][3] = 0.f;
-  R.m0 = R.m1 = -INFINITY;
-  R.l0 = R.l1 = 0.f;
-  const float c = a.scale_log2;
-  const int W = a.window;
-
-  for (int t = 0; t < n_blocks; ++t) {
-    const int s = t % kStages;
-    if (issuer && t > 0 && issued < n_blocks) {
-      // every warp has released step t - 1's stage: refill it
-      if (!mbar_wait(&sm.empty[(t - 1) % kStages], ((t - 1) / kStages) & 1, abort_flag)) {
-        record_error(kErrDecodeMq + 1);
-        *abort_flag = 1;
-      } else {
-        issue(issued++);
+  if (warp == 2) {
+    // ---------------------------------------------------- Q and K producer
+    if (lane == 0) {
+      prefetch_tensormap(&q_map);
+      prefetch_tensormap(&k_map);
+      mbar_arrive_expect_tx(&sm.q_full, 2u * 128u * (uint32_t)n_rows);
+      tma_load_4d(sm.q, &q_map, &sm.q_full, 0, kvh * G, 0, b);
+      tma_load_4d(sm.q + kBoxBytes, &q_map, &sm.q_full, 64, kvh * G, 0, b);
+      int issued = 0;
+      for (int j = 0; j < n_tot; ++j) {
+        const int st = j % kKStages;
+        if (j >= kKStages && !mbar_wait_sleep(&sm.k_empty[st], (j / kKStages - 1) & 1, abort_flag, 256)) {
+          fail(abort_flag, kErrDecodeMq + 1);
+          break;
+        }
+        if (j < n_cb) {
+          const int key0 = k_begin + j * KB;
+          mbar_arrive_expect_tx(&sm.k_full[st], kBlockBytes);
+          tma_load_3d(sm.k[st], &k_map, &sm.k_full[st], 0, key0, row3);
+          tma_load_3d(sm.k[st] + kBoxBytes, &k_map, &sm.k_full[st], 64, key0, row3);
+        } else {
+          mbar_arrive_expect_tx(&sm.k_full[st], 2 * kNewBoxBytes);
+          tma_load_4d(sm.k[st], &kn_map, &sm.k_full[st], 0, kvh, 0, b);
+          tma_load_4d(sm.k[st] + kBoxBytes, &kn_map, &sm.k_full[st], 64, kvh, 0, b);
+        }
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait(&sm.q_full, 0, nullptr, 200000000ull);
+        for (int j = issued > kKStages ? issued - kKStages : 0; j < issued; ++j)
+          mbar_wait(&sm.k_full[j % kKStages], (j / kKStages) & 1, nullptr, 200000000ull);
       }
     }
-    if (*abort_flag || !mbar_wait(&sm.full[s], (t / kStages) & 1, abort_flag)) {
-      record_error(kErrDecodeMq + 2);
-      *abort_flag = 1;
-      break;
+  } else if (warp == 4) {
+    // ---------------------------------------------------------- V producer
+    if (lane == 0) {
+      prefetch_tensormap(&v_map);
+      int issued = 0;
+      for (int j = 0; j < n_tot; ++j) {
+        const int st = j % kVStages;
+        if (j >= kVStages && !mbar_wait_sleep(&sm.v_empty[st], (j / kVStages - 1) & 1, abort_flag, 256)) {
+          fail(abort_flag, kErrDecodeMq + 5);
+          break;
+        }
+        if (j < n_cb) {
+          const int key0 = k_begin + j * KB;
+          mbar_arrive_expect_tx(&sm.v_full[st], kBlockBytes);
+          tma_load_3d(sm.v[st], &v_map, &sm.v_full[st], 0, key0, row3);
+          tma_load_3d(sm.v[st] + kBoxBytes, &v_map, &sm.v_full[st], 64, key0, row3);
+        } else {
+          mbar_arrive_expect_tx(&sm.v_full[st], 2 * kNewBoxBytes);
+          tma_load_4d(sm.v[st], &vn_map, &sm.v_full[st], 0, kvh, 0, b);
+          tma_load_4d(sm.v[st] + kBoxBytes, &vn_map, &sm.v_full[st], 64, kvh, 0, b);
+        }
+        issued = j + 1;
+      }
+      if (*abort_flag)
+        for (int j = issued > kVStages ? issued - kVStages : 0; j < issued; ++j)
+          mbar_wait(&sm.v_full[j % kVStages], (j / kVStages) & 1, nullptr, 200000000ull);
     }
-    const uint32_t kbase = smem_u32(sm.stage[s]);
-    const uint32_t vbase = kbase + 2 * kBoxBytes;
-    const int key0 = k_begin + t * KB;
-    const int live = k_end - key0;
-    // A block needs masks when it is ragged or, on a ring, holds one of the
-    // T oldest slots (dist < T): the first key's dist, or the wrap point
-    // (dist 0) inside the block.
-    bool masked = live < KB;
-    if (ring && !masked) {
-      int d_first = key0 - newest - 1;
-      if (d_first < 0) d_first += W;
-      const int wrap = (newest + 1) % W;
-      masked = d_first < T || (wrap > key0 && wrap < key0 + KB);
-    }
-    if (masked) {
-      auto vis = [&](int kidx, int hi) -> bool {
-        if (kidx >= live) return false;
-        if (!ring) return true;
-        int d = key0 + kidx - newest - 1;
-        if (d < 0) d += W;
-        return d > (hi ? t1 : t0);
+  } else if (warp == 3) {
+    // ----------------------------------------------------------- MMA issuer
+    // QK^T(j) into S[j & 1], then P(j - 1).V: the QK^T of a block overlaps the
+    // softmax of the previous one.  QK^T(j) overwrites the columns of P(j - 2)
+    // only after P(j - 2).V, issued before it, has read them.
+    if (lane == 0) {
+      const uint64_t qd = sw128_desc(smem_u32(sm.q), 16, 1024);
+      const uint64_t kd = sw128_desc(smem_u32(sm.k[0]), 16, 1024);
+      const uint64_t vd = sw128_desc(smem_u32(sm.v[0]), kBoxBytes, 1024);
+      const uint32_t idesc_qk = idesc_bf16_f32(128, KB, false, false);
+      const uint32_t idesc_qk_new = idesc_bf16_f32(128, kNewRows, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
+      int issued_pv = 0;
+      auto pv = [&](int x) -> bool {
+        if (!mbar_wait(&sm.p_full[x & 1], (x >> 1) & 1, abort_flag) ||
+            !mbar_wait(&sm.v_full[x % kVStages], (x / kVStages) & 1, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t b0 = (uint32_t)vd + (uint32_t)(((x % kVStages) * kBlockBytes) >> 4);
+        const int n_k16 = x < n_cb ? KB / 16 : 1;
+        for (int kk = 0; kk < n_k16; ++kk)
+          umma_ts_lh(tmem + 128, tmem + (x & 1) * 64 + kk * 8, b0 + (uint32_t)((kk * 2048) >> 4),
+                     (uint32_t)(vd >> 32), idesc_pv, (x > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&sm.v_empty[x % kVStages]);
+        umma_commit(&sm.pv_done[x & 1]);
+        issued_pv = x + 1;
+        return true;
       };
-      mq_block<KB, true>(R, kbase, vbase, kBoxBytes, c, lane, live, dead_slot < 0 ? -1 : dead_slot - key0, vis);
-    } else {
-      mq_block<KB, false>(R, kbase, vbase, kBoxBytes, c, lane, KB, -1, [](int, int) -> bool { return true; });
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.empty[s]);
-  }
-  __syncthreads();  // every warp is past the loop, aborted or not
-  if (*abort_flag) {
-    // let every copy the issuer started land before the CTA exits
-    if (issuer)
-      for (int t = issued > kStages ? issued - kStages : 0; t < issued; ++t)
-        mbar_wait(&sm.full[t % kStages], (t / kStages) & 1, nullptr, 200000000ull);
-    return;
-  }
-
-  if (has_new) {
-    // every warp is past its last stage read and every load has landed:
-    // stage 0 takes the new tokens' K and V rows (zero past T)
-    for (int i = threadIdx.x; i < 2 * kNewRows * 16; i += MT * 32) {
-      const int tensor = i / (kNewRows * 16), row = (i >> 4) % kNewRows, ch = i & 15;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row < T) {
-        const uint16_t* src = (tensor ? a.v_new : a.k_new) + (((size_t)b * T + row) * a.Hkv + kvh) * kHeadDim;
-        v = __ldg(reinterpret_cast<const uint4*>(src) + ch);
+      for (int j = 0; j < n_tot && ok; ++j) {
+        ok = mbar_wait(&sm.k_full[j % kKStages], (j / kKStages) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t b0 = (uint32_t)kd + (uint32_t)(((j % kKStages) * kBlockBytes) >> 4);
+        const uint32_t idesc = j < n_cb ? idesc_qk : idesc_qk_new;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (uint32_t)((((kk >> 2) * kBoxBytes) + (kk & 3) * 32) >> 4);
+          umma_ss_lh(tmem + (j & 1) * 64, (uint32_t)qd + off, (uint32_t)(qd >> 32), b0 + off, (uint32_t)(kd >> 32),
+                     idesc, kk > 0);
+        }
+        umma_commit(&sm.s_full[j & 1]);
+        umma_commit(&sm.k_empty[j % kKStages]);
+        if (j > 0) ok = pv(j - 1);
       }
-      *reinterpret_cast<uint4*>(sm.stage[0] + (tensor * 2 + (ch >> 3)) * kBoxBytes + sw128_off(row, ch & 7)) = v;
+      if (ok) ok = pv(n_tot - 1);
+      if (!ok) fail(abort_flag, kErrDecodeMq + 6);
+      (void)issued_pv;
+      // every MMA of this thread completes before the CTA moves on
+      umma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, nullptr, 200000000ull);
     }
-    __syncthreads();
-    const uint32_t fb = smem_u32(sm.stage[0]);
-    auto vis = [&](int j, int hi) -> bool {
-      const int tq = hi ? t1 : t0;
-      return j <= tq && (!ring || j > tq - W);
-    };
-    mq_block<kNewRows, true>(R, fb, fb + 2 * kBoxBytes, kBoxBytes, c, lane, kNewRows, -1, vis);
+  } else if (warp < 2) {
+    // ------------------------------------------------ softmax (thread = row)
+    const int r = threadIdx.x;  // 0..63
+    const bool valid = r < n_rows;
+    const int t = valid ? r / G : 0;
+    const int hq = kvh * G + (valid ? r % G : 0);
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float c = a.scale_log2;
+    const int W = a.window;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tot; ++j) {
+      const bool is_new = j >= n_cb;
+      const int key0 = k_begin + j * KB;
+      const int live = is_new ? T : k_end - key0;  // keys of the block that exist
+      if (!warp_wait(&sm.s_full[j & 1], (j >> 1) & 1, abort_flag)) {
+        fail(abort_flag, kErrDecodeMq + 2);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + (j & 1) * 64;
+      uint32_t v[64];
+      if (!is_new) {
+        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      } else {
+        tmem_ld16(s_addr, *reinterpret_cast<uint32_t(*)[16]>(v));
+      }
+      tmem_wait_ld();
+      // A cache block needs per-key masks only when it is ragged or, on a
+      // ring, holds one of the T oldest slots (ring distance < T); the rows past
+      // T * G read zero queries and need none.  Scores are kept unscaled
+      // (raw dot products); the scale goes into the exponent.
+      const int dbase = key0 - newest - 1;  // ring distance of key 0 of the block, unwrapped
+      const int d0 = dbase < 0 ? dbase + W : dbase;
+      const bool masked = is_new || live < KB || (ring && (d0 < T || (dbase < 0 && dbase + KB > 0)));
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (is_new) {
+#pragma unroll
+        for (int e = 0; e < kNewRows; ++e) {
+          const bool vis = e < live && e <= t && (!ring || e > t - W);
+          if (!vis) v[e] = __float_as_uint(-INFINITY);
+          mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
+        }
+      } else if (masked) {
+#pragma unroll
+        for (int e = 0; e < KB; ++e) {
+          int dd = dbase + e;
+          dd += dd < 0 ? W : 0;
+          const bool vis = e < live && (!ring || dd > t);
+          if (!vis) v[e] = __float_as_uint(-INFINITY);
+          mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e]));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < KB; e += 2)
+          mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+      }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+      const float m_use = (mt - m > 8.f) ? mt : m;  // lazy: the max moves only by more than 8
+      const float m_safe = m_use == -INFINITY ? 0.f : m_use;
+      const float alpha = fast_exp2(m - m_safe);
+      float sum = 0.f;
+      uint32_t pk[32];
+      if (is_new) {
+#pragma unroll
+        for (int e = 0; e < kNewRows; e += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(v[e]), c, -m_safe));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(v[e + 1]), c, -m_safe));
+          sum += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+      } else {
+        const uint64_t cc = f2_pack(c, c), mm = f2_pack(-m_safe, -m_safe);
+        uint64_t s2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int e = 0; e < KB; e += 2) {
+          const uint64_t y = f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), cc, mm);
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+          s2[(e >> 1) & 3] = f2_add(s2[(e >> 1) & 3], f2_pack(p0, p1));
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(s2[0], s2[1]), f2_add(s2[2], s2[3])), a0, a1);
+        sum = a0 + a1;
+      }
+      // P over the S columns it came from
+      if (!is_new) {
+        tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+      } else {
+        tmem_st8(s_addr, pk);
+      }
+      // keys no row sees (past the live end; a full ring's oldest slot) may
+      // hold NaN: zero their V rows before P.V, which multiplies them by 0
+      const int dead = (ring && L0 >= W && !is_new) ? (newest + 1) % W - key0 : -1;
+      const bool ragged = !is_new && live < KB;
+      const bool dead_in = (unsigned)dead < (unsigned)KB;
+      if (ragged || dead_in) {
+        if (!warp_wait(&sm.v_full[j % kVStages], (j / kVStages) & 1, abort_flag)) {
+          fail(abort_flag, kErrDecodeMq + 7);
+          ok = false;
+          break;
+        }
+        uint8_t* vst = sm.v[j % kVStages];
+        // thread r zeroes key row r (64 rows, 64 threads)
+        if (r >= live || r == dead) {
+#pragma unroll
+          for (int ch = 0; ch < 16; ++ch)
+            *reinterpret_cast<uint4*>(vst + (ch >> 3) * kBoxBytes + sw128_off(r, ch & 7)) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      // O holds blocks 0..j-1: bring it to the new max before P(j).V adds to it
+      // (a row that has seen no key yet holds O = 0 and needs nothing)
+      if (j > 0 && __any_sync(0xffffffffu, valid && m != -INFINITY && alpha != 1.f)) {
+        if (!warp_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
+          fail(abort_flag, kErrDecodeMq + 8);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t o_addr = tmem + lane_base + 128;
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + q4 * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(o_addr + q4 * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[j & 1]);
+      l = l * alpha + sum;
+      m = m_use;
+    }
+    // ---- result: the last P.V complete, then O of this row
+    if (ok && warp_wait(&sm.pv_done[(n_tot - 1) & 1], ((n_tot - 1) >> 1) & 1, abort_flag)) {
+      tc_fence_after();
+      const uint32_t o_addr = tmem + lane_base + 128;
+      const size_t row = ((size_t)b * T + t) * a.Hq + hq;
+      const float f = (a.max_splits == 1) ? (a.gate ? sigmoidf_(a.gate[row]) : 1.f) / l : 1.f;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t o[32];
+        tmem_ld32(o_addr + q4 * 32, o);
+        tmem_wait_ld();
+        if (valid) {
+          if (a.max_splits == 1) {
+            uint4* dst = reinterpret_cast<uint4*>(a.out + row * kHeadDim) + q4 * 4;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+              dst[c4] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * c4]) * f, __uint_as_float(o[8 * c4 + 1]) * f),
+                                   pack_bf16x2(__uint_as_float(o[8 * c4 + 2]) * f, __uint_as_float(o[8 * c4 + 3]) * f),
+                                   pack_bf16x2(__uint_as_float(o[8 * c4 + 4]) * f, __uint_as_float(o[8 * c4 + 5]) * f),
+                                   pack_bf16x2(__uint_as_float(o[8 * c4 + 6]) * f, __uint_as_float(o[8 * c4 + 7]) * f));
+          } else {
+            const size_t slot = row * a.max_splits + split;
+            float4* dst = reinterpret_cast<float4*>(a.part_o + slot * kHeadDim) + q4 * 8;
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+              dst[c4] = make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
+                                    __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
+            if (q4 == 0) a.part_ml[slot] = make_float2(m, l);
+          }
+        }
+      }
+    } else if (ok) {
+      fail(abort_flag, kErrDecodeMq + 9);
+    }
   }
 
-  float l0 = R.l0, l1 = R.l1;
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  if (a.max_splits == 1) {
-    if (v0) {
-      const float sc = (a.gate ? sigmoidf_(a.gate[row0]) : 1.f) / l0;
-      uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + row0 * kHeadDim);
-#pragma unroll
-      for (int n = 0; n < 16; ++n) dst[n * 4 + tig] = pack_bf16x2(R.o[n][0] * sc, R.o[n][1] * sc);
-    }
-    if (v1) {
-      const float sc = (a.gate ? sigmoidf_(a.gate[row1]) : 1.f) / l1;
-      uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + row1 * kHeadDim);
-#pragma unroll
-      for (int n = 0; n < 16; ++n) dst[n * 4 + tig] = pack_bf16x2(R.o[n][2] * sc, R.o[n][3] * sc);
-    }
-  } else {
-    if (v0) {
-      const size_t slot = row0 * a.max_splits + split;
-      float2* dst = reinterpret_cast<float2*>(a.part_o + slot * kHeadDim);
-#pragma unroll
-      for (int n = 0; n < 16; ++n) dst[n * 4 + tig] = make_float2(R.o[n][0], R.o[n][1]);
-      if (tig == 0) a.part_ml[slot] = make_float2(R.m0, l0);
-    }
-    if (v1) {
-      const size_t slot = row1 * a.max_splits + split;
-      float2* dst = reinterpret_cast<float2*>(a.part_o + slot * kHeadDim);
-#pragma unroll
-      for (int n = 0; n < 16; ++n) dst[n * 4 + tig] = make_float2(R.o[n][2], R.o[n][3]);
-      if (tig == 0) a.part_ml[slot] = make_float2(R.m1, l1);
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -387,33 +488,24 @@ __global__ void __launch_bounds__(128) decode_mq_combine_kernel(const DecodeMqAr
   a.out[row * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(acc / lsum * gt));
 }
 
-template <int MT>
-cudaError_t launch_mq(const DecodeMqArgs& a, const CUtensorMap& k_map, const CUtensorMap& v_map,
-                      cudaStream_t stream) {
-  const size_t smem = sizeof(MqSmem) + 1024;
-  static DeviceOnce setup;
-  cudaError_t e = device_once(setup, [&](int, int*) {
-    return cudaFuncSetAttribute(decode_mq_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  });
-  if (e != cudaSuccess) return e;
-  e = launch_kernel(true, decode_mq_kernel<MT>, dim3(a.max_splits, a.Hkv, a.B), dim3(MT * 32), smem, stream, a, k_map,
-                       v_map);
-  if (e != cudaSuccess || a.max_splits == 1) return e;
-  return launch_kernel(true, decode_mq_combine_kernel, dim3(a.Hq, a.T, a.B), dim3(kHeadDim), 0, stream, a);
-}
-
 }  // namespace decode_mq_detail
 
-cudaError_t launch_decode_mq(const DecodeMqArgs& a, const CUtensorMap& k_map, const CUtensorMap& v_map,
+cudaError_t launch_decode_mq(const DecodeMqArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
+                             const CUtensorMap& v_map, const CUtensorMap& kn_map, const CUtensorMap& vn_map,
                              cudaStream_t stream) {
+  using namespace decode_mq_detail;
   if (a.B == 0) return cudaSuccess;
-  switch ((a.T * a.G + 15) / 16) {
-    case 1: return decode_mq_detail::launch_mq<1>(a, k_map, v_map, stream);
-    case 2: return decode_mq_detail::launch_mq<2>(a, k_map, v_map, stream);
-    case 3: return decode_mq_detail::launch_mq<3>(a, k_map, v_map, stream);
-    case 4: return decode_mq_detail::launch_mq<4>(a, k_map, v_map, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  const size_t smem = sizeof(Smem) + 1024;
+  static DeviceOnce setup;
+  cudaError_t e = device_once(setup, [&](int, int*) {
+    return cudaFuncSetAttribute(decode_mq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
+  if (e != cudaSuccess) return e;
+  e = launch_kernel(true, decode_mq_kernel, dim3(a.max_splits, a.Hkv, a.B), dim3(kThreads), smem, stream, a,
+                    q_map, k_map, v_map, kn_map, vn_map);
+  if (e != cudaSuccess || a.max_splits == 1) return e;
+  return launch_kernel(true, decode_mq_combine_kernel, dim3(a.Hq, a.T, a.B), dim3(kHeadDim), 0,
+                       stream, a);
 }
 
 }  // namespace swa

@@ -230,11 +230,10 @@ DecodePlan plan_decode(const swa_layer_params* p, int B, int max_len) {
 // tokens ride on the last split), with the kernel's resident CTAs per SM.
 DecodePlan plan_decode_mq(const swa_layer_params* p, int B, int T, int max_len) {
   DecodePlan pl{};
-  const long long kb = swa::kDecodeKeyBlock;
+  const long long kb = swa::kDecodeMqKeyBlock;
   const long long ctx = max_len - T > 0 ? max_len - T : 0;
   const long long n_vis = p->window > 0 ? (ctx < p->window ? ctx : p->window) : ctx;
-  const int rows = T * (p->num_q_heads / p->num_kv_heads);
-  const long long slots = 148LL * swa::decode_mq_ctas_per_sm(rows), items = (long long)B * p->num_kv_heads;
+  const long long slots = 148LL * swa::kDecodeMqCtasPerSm, items = (long long)B * p->num_kv_heads;
   long long c = (items * n_vis + slots - 1) / slots;
   c = (c + kb - 1) / kb * kb;
   if (c < 256) c = 256;
@@ -632,9 +631,26 @@ swa_status swa_attn_decode_mq(const swa_layer_params* p, int32_t B, int32_t T, c
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
       return fail(SWA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   }
-  CUtensorMap km, vm;
-  if ((st = encode_cache(&km, k_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
-  if ((st = encode_cache(&vm, v_cache, B * Hkv, cache_capacity, swa::kDecodeKeyBlock)) != SWA_OK) return st;
+  // q [B, T, Hq, D] -> {D, Hq, T, B}, box {64, G, T, 1}: the (t, g) rows of one kv-head
+  // k_new / v_new [B, T, Hkv, D] -> {D, Hkv, T, B}, box {64, 1, 16, 1} (rows past T read as zero)
+  CUtensorMap qm, km, vm, knm, vnm;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)Hq * kHeadDim * 2,
+                                   (cuuint64_t)T * Hq * kHeadDim * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)T, 1};
+    if ((st = encode_bf16(&qm, q, 4, dims, strides, box)) != SWA_OK) return st;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hkv, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)Hkv * kHeadDim * 2,
+                                   (cuuint64_t)T * Hkv * kHeadDim * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)swa::kDecodeMqMaxT, 1};
+    if ((st = encode_bf16(&knm, k_new, 4, dims, strides, box)) != SWA_OK) return st;
+    if ((st = encode_bf16(&vnm, v_new, 4, dims, strides, box)) != SWA_OK) return st;
+  }
+  if ((st = encode_cache(&km, k_cache, B * Hkv, cache_capacity, swa::kDecodeMqKeyBlock)) != SWA_OK) return st;
+  if ((st = encode_cache(&vm, v_cache, B * Hkv, cache_capacity, swa::kDecodeMqKeyBlock)) != SWA_OK) return st;
   swa::DecodeMqArgs a{};
   a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.window = p->window; a.capacity = cache_capacity;
   a.scale_log2 = scale_log2(p);
@@ -642,7 +658,7 @@ swa_status swa_attn_decode_mq(const swa_layer_params* p, int32_t B, int32_t T, c
   a.chunk = pl.chunk; a.max_splits = pl.splits;
   a.part_o = pl.splits > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
   a.part_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace) + pl.o_bytes) : nullptr;
-  st = cuda_status(swa::launch_decode_mq(a, km, vm, (cudaStream_t)stream), "multi-query decode launch");
+  st = cuda_status(swa::launch_decode_mq(a, qm, km, vm, knm, vnm, (cudaStream_t)stream), "multi-query decode launch");
   return st == SWA_OK ? ok() : st;
 }
 

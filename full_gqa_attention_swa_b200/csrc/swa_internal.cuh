@@ -177,8 +177,6 @@ constexpr int kDecodeKeyBlock = 32;   // keys per pipeline stage
 
 constexpr int kDecodeMqMaxT = 16;      // new tokens per sequence
 constexpr int kDecodeMqMaxRows = 64;   // T * G (query, head) rows per kv-head
-// resident multi-query decode CTAs per SM for T * G rows (sizes the split plan)
-constexpr int decode_mq_ctas_per_sm(int rows) { return rows <= 48 ? 4 : 3; }
 
 struct DecodeMqArgs {
   int B, T, Hq, Hkv, G;
@@ -197,8 +195,14 @@ struct DecodeMqArgs {
   float2* part_ml;           // [B*T*Hq][max_splits]
 };
 
-// kv maps as for launch_decode; m_tiles = ceil(T*G / 16) selects the kernel.
-cudaError_t launch_decode_mq(const DecodeMqArgs& a, const CUtensorMap& k_map, const CUtensorMap& v_map,
+// q_map 4-D {D, Hq, T, B} box {64, G, T, 1} (the (t, g) rows of one kv-head);
+// k_map / v_map 3-D {D, C, B*Hkv} box {64, 64, 1}; kn_map / vn_map (the new
+// tokens' keys and values) 4-D {D, Hkv, T, B} box {64, 1, 16, 1}; chunk a
+// multiple of kDecodeMqKeyBlock.
+constexpr int kDecodeMqKeyBlock = 64;
+constexpr int kDecodeMqCtasPerSm = 2;
+cudaError_t launch_decode_mq(const DecodeMqArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
+                             const CUtensorMap& v_map, const CUtensorMap& kn_map, const CUtensorMap& vn_map,
                              cudaStream_t stream);
 
 }  // namespace swa
