@@ -431,8 +431,9 @@ swa_status swa_attn_prefill(const swa_layer_params* p, int32_t B, int32_t S, con
     if (st != SWA_OK) return st;
     k_att = k_rot;
   }
-  CUtensorMap qm, km, vm;
+  CUtensorMap qm, km, vm, om;
   if ((st = encode_bshd(&qm, q, B, S, Hq, 128)) != SWA_OK) return st;
+  if ((st = encode_bshd(&om, out, B, S, Hq, 128)) != SWA_OK) return st;
   if ((st = encode_bshd(&km, k_att, B, S, Hkv, 128)) != SWA_OK) return st;
   if ((st = encode_bshd(&vm, v, B, S, Hkv, 128)) != SWA_OK) return st;
   swa::PrefillArgs a{};
@@ -443,8 +444,7 @@ swa_status swa_attn_prefill(const swa_layer_params* p, int32_t B, int32_t S, con
   a.gate = gate;
   a.n_q_tiles = (int)n_q_tiles;
   a.n_head_pairs = (G + 1) / 2;
-  a.out = out;
-  st = cuda_status(swa::launch_prefill(a, qm, km, vm, s), "prefill launch");
+  st = cuda_status(swa::launch_prefill(a, qm, km, vm, om, s), "prefill launch");
   return st == SWA_OK ? ok() : st;
 }
 
@@ -514,8 +514,9 @@ swa_status swa_attn_prefill_chunk(const swa_layer_params* p, int32_t B, int32_t 
   st = cuda_status(swa::launch_rope(r, s), "rope (chunk keys) launch");
   if (st != SWA_OK) return st;
 
-  CUtensorMap qm, km, vm;
+  CUtensorMap qm, km, vm, om;
   if ((st = encode_bshd(&qm, q, B, S, Hq, 128)) != SWA_OK) return st;
+  if ((st = encode_bshd(&om, out, B, S, Hq, 128)) != SWA_OK) return st;
   swa::PrefillArgs a{};
   if (pl.ring) {
     if ((st = encode_bshd(&km, k_seq, B, pl.h + S, Hkv, 128)) != SWA_OK) return st;
@@ -535,8 +536,7 @@ swa_status swa_attn_prefill_chunk(const swa_layer_params* p, int32_t B, int32_t 
   a.gate = gate;
   a.n_q_tiles = (int)n_q_tiles;
   a.n_head_pairs = (G + 1) / 2;
-  a.out = out;
-  st = cuda_status(swa::launch_prefill(a, qm, km, vm, s), "prefill (chunk) launch");
+  st = cuda_status(swa::launch_prefill(a, qm, km, vm, om, s), "prefill (chunk) launch");
   return st == SWA_OK ? ok() : st;
 }
 

@@ -33,7 +33,8 @@
 //               O row when the running max moves (rare: lazy threshold)
 //   warps 4-7   head slot 1 softmax
 //   warps 8-11  next tile's Q rotation, then this tile's epilogue
-//               (O / l * sigmoid(gate) -> bf16 -> global, thread = row)
+//               (O / l * sigmoid(gate) -> bf16, thread = row, staged in the
+//               tile's own Q buffers and written by TMA stores)
 //   warp 12     tcgen05.mma issuer (one thread)
 //   warp 13     K / V TMA producer (one thread), three-stage ring
 //   warp 15     Q TMA producer (one thread)
@@ -72,13 +73,14 @@ struct Smem {
   uint8_t kv[kKvStages][kTileBytes];
   float lsum[2][2][BM];            // [tile parity][head slot][row]: softmax row sums
   uint64_t q_full[2][2];           // Q of [parity][slot] landed
-  uint64_t q_empty[2][2];          // the last QK^T reading Q[parity][slot] completed
+  uint64_t q_free[2];              // the output staged in Q[parity][*] has been read by its TMA store
   uint64_t q_ready[2];             // both slots' Q rotated (128 arrivals)
   uint64_t kv_full[kKvStages], kv_empty[kKvStages];
   uint64_t s_full[2];              // S_s complete (and every earlier MMA, P_s.V included)
   uint64_t p_full[2];              // P_s written, O_s rescaled (128 arrivals)
   uint64_t o_done[2];              // the tile's last P_s.V complete
   uint64_t o_free[2];              // the epilogue has read O_s (128 arrivals)
+  uint64_t o_staged[2];            // the bf16 output of slot s is in shared memory (128 arrivals)
   uint64_t l_full[2][2];           // [parity][slot] row sums written (128 arrivals)
   uint64_t drain;
   uint32_t tmem_base;
@@ -182,7 +184,8 @@ __device__ __forceinline__ void rotate_q_row_scalar(uint8_t* tile, int row, int 
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap q_map,
-                   const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map) {
+                   const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
+                   const __grid_constant__ CUtensorMap o_map) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need 1024-byte alignment and the layout has
   // no room to realign: leave (uniformly, before any barrier) if it is off
@@ -198,10 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       for (int s = 0; s < 2; ++s) {
         mbar_init(&sm.q_full[b][s], 1);
-        mbar_init(&sm.q_empty[b][s], 1);
         mbar_init(&sm.l_full[b][s], BM);
       }
       mbar_init(&sm.q_ready[b], BM);
+      mbar_init(&sm.q_free[b], 1);
     }
     for (int i = 0; i < kKvStages; ++i) {
       mbar_init(&sm.kv_full[i], 1);
@@ -212,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[s], BM);
       mbar_init(&sm.o_done[s], 1);
       mbar_init(&sm.o_free[s], BM);
+      mbar_init(&sm.o_staged[s], BM);
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -268,19 +272,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 15 && lane == 0) {
       // ========================================================== Q producer
-      // Q of tile it goes to buffer it & 1 once the last QK^T of tile it - 2
-      // (the buffer's previous tile) has completed.
+      // Q of tile it goes to buffer it & 1 once the output of tile it - 2
+      // (the buffer's previous tile), staged there by the epilogue, has been
+      // read by its TMA store.
       prefetch_tensormap(&q_map);
       int it = 0, last_it = -1;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
         const Tile N = decode_tile<kMode>(a, t);
         const int b = it & 1;
+        if (it >= 2 && !mbar_wait(&sm.q_free[b], ((it - 2) >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
         for (int s = 0; s < 2; ++s) {
-          if (it >= 2 && !mbar_wait(&sm.q_empty[b][s], ((it - 2) >> 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
           const int h = s ? N.h1 : N.h0;
           mbar_arrive_expect_tx(&sm.q_full[b][s], kTileBytes);
           tma_load_4d(sm.q[b][s], &q_map, &sm.q_full[b][s], 0, h, N.r0, N.b);
@@ -339,7 +344,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int s = 0; s < 2; ++s) {
             issue_qk(0, s, 0);
             umma_commit(&sm.s_full[s]);
-            if (T0.n_kv == 1) umma_commit(&sm.q_empty[0][s]);
           }
           umma_commit(&sm.kv_empty[0]);
         } else {
@@ -349,7 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
         const int n = decode_tile<kMode>(a, t).n_kv;
         const bool has_next = t + (int)gridDim.x < n_tiles;
-        const int n_next = has_next ? decode_tile<kMode>(a, t + gridDim.x).n_kv : 0;
         const int b = it & 1, nb = b ^ 1;
         for (int j = 0; j < n && ok; ++j) {
           const bool last = j == n - 1;
@@ -378,9 +381,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               issue_qk(last ? nb : b, s, kidx);
               umma_commit(&sm.s_full[s]);
               if (s == 1) umma_commit(&sm.kv_empty[kidx % kKvStages]);
-              // the last QK^T that reads this Q buffer frees it for a later tile
-              if (!last && j + 2 == n) umma_commit(&sm.q_empty[b][s]);
-              if (last && n_next == 1) umma_commit(&sm.q_empty[nb][s]);
             }
           }
         }
@@ -456,7 +456,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
         const float m_use = (mt - m > kRescaleThreshold) ? mt : m;  // m = -inf: always take mt
         const float m_safe = m_use == -INFINITY ? 0.f : m_use;
-        const float alpha = fast_exp2(m - m_safe);
+        // a row that has seen no visible key yet has O = 0 and l = 0: it
+        // needs no rescale (alpha 1 keeps the band-edge tile's emptiest row
+        // from sending its whole warp through the O rescale)
+        const float alpha = m == -INFINITY ? 1.f : fast_exp2(m - m_safe);
         // P = 2^(c S - m), two columns per packed FMA; masked columns give 0
         const uint64_t cc = f2_pack(c, c), mm = f2_pack(-m_safe, -m_safe);
         uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
@@ -576,20 +579,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         fail(abort_flag, kErrPrefill + 8);
         break;
       }
-      // ---- epilogue: out = O / l * sigmoid(gate), bf16, straight to global
+      // ---- epilogue: out = O / l * sigmoid(gate), bf16, staged in this
+      // tile's Q buffers (their last QK^T completed before O did) and
+      // written by TMA stores; the Q producer refills the buffers once the
+      // stores have read them
+      const int b = it & 1;
       for (int s = 0; s < 2 && ok; ++s) {
         if (!warp_wait(&sm.o_done[s], it & 1, abort_flag) ||
-            !warp_wait(&sm.l_full[it & 1][s], (it >> 1) & 1, abort_flag)) {
+            !warp_wait(&sm.l_full[b][s], (it >> 1) & 1, abort_flag)) {
           fail(abort_flag, kErrPrefill + 11);
           ok = false;
           break;
         }
         tc_fence_after();
-        const float l = sm.lsum[it & 1][s][row];
+        const float l = sm.lsum[b][s][row];
         const float gt = a.gate ? 1.f / (1.f + __expf(-(s ? glog1 : glog0))) : 1.f;
         const float f = gt / l;
-        const bool store = r < a.S && (s == 0 || T.store1);
-        uint4* dst = reinterpret_cast<uint4*>(a.out + (((size_t)T.b * a.S + r) * a.Hq + (s ? T.h1 : T.h0)) * 128);
+        uint8_t* stage = sm.q[b][s];
         const uint32_t oaddr = tmem + lane_base + 256 + s * 128;
 #pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -601,20 +607,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&sm.o_free[s]);
           }
-          if (store) {
+          uint8_t* box = stage + (q4 >> 1) * kBoxBytes;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(v[8 * c4 + 0]) * f, __uint_as_float(v[8 * c4 + 1]) * f);
-              u.y = pack_bf16x2(__uint_as_float(v[8 * c4 + 2]) * f, __uint_as_float(v[8 * c4 + 3]) * f);
-              u.z = pack_bf16x2(__uint_as_float(v[8 * c4 + 4]) * f, __uint_as_float(v[8 * c4 + 5]) * f);
-              u.w = pack_bf16x2(__uint_as_float(v[8 * c4 + 6]) * f, __uint_as_float(v[8 * c4 + 7]) * f);
-              dst[q4 * 4 + c4] = u;
-            }
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(v[8 * c4 + 0]) * f, __uint_as_float(v[8 * c4 + 1]) * f);
+            u.y = pack_bf16x2(__uint_as_float(v[8 * c4 + 2]) * f, __uint_as_float(v[8 * c4 + 3]) * f);
+            u.z = pack_bf16x2(__uint_as_float(v[8 * c4 + 4]) * f, __uint_as_float(v[8 * c4 + 5]) * f);
+            u.w = pack_bf16x2(__uint_as_float(v[8 * c4 + 6]) * f, __uint_as_float(v[8 * c4 + 7]) * f);
+            *reinterpret_cast<uint4*>(box + sw128_off(row, (q4 & 1) * 4 + c4)) = u;
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.o_staged[s]);
+        if (threadIdx.x == 256) {
+          // one thread stores the tile (rows at or beyond S are clipped by
+          // the tensor map); a time-out only records the error and sets the
+          // abort flag, so that the warp's lanes stay on one path
+          if (!mbar_wait(&sm.o_staged[s], it & 1, abort_flag)) {
+            fail(abort_flag, kErrPrefill + 12);
+          } else if (s == 0 || T.store1) {
+            const int h = s ? T.h1 : T.h0;
+            tma_store_4d(&o_map, stage, 0, h, T.r0, T.b);
+            tma_store_4d(&o_map, stage + kBoxBytes, 64, h, T.r0, T.b);
+            bulk_commit_group();
           }
         }
       }
+      if (threadIdx.x == 256) {
+        bulk_wait_group_read0();
+        mbar_arrive(&sm.q_free[b]);
+      }
     }
+    // the output stores complete before the CTA exits
+    if (threadIdx.x == 256) bulk_wait_group0();
   }
 
   tc_fence_before();
@@ -627,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int kMode>
 cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                             const CUtensorMap& v_map, cudaStream_t stream) {
+                             const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream) {
   const long long n_tiles = (long long)a.n_q_tiles * a.n_head_pairs * a.Hkv * a.B;
   if (n_tiles == 0) return cudaSuccess;
   if (n_tiles > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
@@ -649,17 +675,17 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& q_map, con
   if (e != cudaSuccess) return e;
   const int grid = (int)(n_tiles < n_sm ? n_tiles : n_sm);
   return launch_kernel(false, prefill_kernel<kMode>, dim3(grid), dim3(kThreads), smem, stream, a, q_map, k_map,
-                       v_map);
+                       v_map, o_map);
 }
 
 }  // namespace prefill_detail
 
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                            const CUtensorMap& v_map, cudaStream_t stream) {
+                            const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream) {
   using namespace prefill_detail;
-  if (a.kv_cache_layout) return launch_prefill_t<kChunkCache>(a, q_map, k_map, v_map, stream);
-  if (a.q_off) return launch_prefill_t<kChunkSeq>(a, q_map, k_map, v_map, stream);
-  return launch_prefill_t<kWhole>(a, q_map, k_map, v_map, stream);
+  if (a.kv_cache_layout) return launch_prefill_t<kChunkCache>(a, q_map, k_map, v_map, o_map, stream);
+  if (a.q_off) return launch_prefill_t<kChunkSeq>(a, q_map, k_map, v_map, o_map, stream);
+  return launch_prefill_t<kWhole>(a, q_map, k_map, v_map, o_map, stream);
 }
 
 }  // namespace swa

@@ -124,15 +124,15 @@ struct PrefillArgs {
   int n_head_pairs;          // ceil(G / 2)
   int q_off;                 // key-space position of query row 0 (keys 0 .. q_off + S - 1); 0 for a whole prefill
   int kv_cache_layout;       // 0: k/v maps {D, Hkv, keys, B}; 1: a KV cache, maps {D, keys, B * Hkv}
-  uint16_t* out;             // [B, S, Hq, D] bf16
 };
 
-// q_map: 4-D {D, Hq, S, B}; k_map / v_map: 4-D {D, Hkv, q_off + S, B} (any
-// strides: a KV cache [B, Hkv, C, D] is addressed in place); boxes
-// {64, 1, 128, 1}, 128-byte swizzle.  Query row r sits at key-space position
-// q_off + r; the cos/sin table, the gate and the output rows are indexed by r.
+// q_map / o_map (the bf16 output [B, S, Hq, D]): 4-D {D, Hq, S, B}; k_map /
+// v_map: 4-D {D, Hkv, q_off + S, B} (any strides: a KV cache [B, Hkv, C, D]
+// is addressed in place); boxes {64, 1, 128, 1}, 128-byte swizzle.  Query row
+// r sits at key-space position q_off + r; the cos/sin table, the gate and the
+// output rows are indexed by r.
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                           const CUtensorMap& v_map, cudaStream_t stream);
+                           const CUtensorMap& v_map, const CUtensorMap& o_map, cudaStream_t stream);
 
 // ------------------------------------------------------ continued prefill
 
