@@ -127,6 +127,14 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Bits lo .. hi of a 32-bit word (none where hi < lo; bounds outside 0..31
+// are clamped).
+__device__ __forceinline__ uint32_t chunk_keep(int lo, int hi) {
+  const uint32_t to_hi = hi >= 31 ? 0xffffffffu : (hi < 0 ? 0u : (2u << hi) - 1u);  // bits 0 .. hi
+  const uint32_t to_lo = lo <= 0 ? 0u : (lo > 31 ? 0xffffffffu : (1u << lo) - 1u);  // bits 0 .. lo - 1
+  return to_hi & ~to_lo;
+}
+
 __device__ __forceinline__ void fail(volatile int* abort_flag, int code) {
   record_error(code);
   *abort_flag = 1;
@@ -430,17 +438,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool cut_lo = a.window > 0 && key0 < T.i0 + BM - a.window;
         uint32_t masked = 0;  // bit q: chunk q masked for every row of the warp
         if (cut_hi || cut_lo) {
-          const int hi = cut_hi ? i - key0 : BN;                 // columns > hi are masked
-          const int lo = cut_lo ? i - a.window + 1 - key0 : -1;  // columns < lo are masked
+          // this row's visible columns are lo .. hi
+          const int hi = cut_hi ? i - key0 : BN - 1;
+          const int lo = cut_lo ? i - a.window + 1 - key0 : 0;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int c0 = 32 * q;
-            if (__all_sync(0xffffffffu, hi < c0 || lo > c0 + 31)) {
+            const uint32_t keep = chunk_keep(lo - 32 * q, hi - 32 * q);  // bit k: column 32 q + k visible
+            if (__all_sync(0xffffffffu, keep == 0u)) {
               masked |= 1u << q;
-            } else if (!__all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31)) {
+            } else if (!__all_sync(0xffffffffu, keep == 0xffffffffu)) {
 #pragma unroll
-              for (int e = c0; e < c0 + 32; ++e)
-                if (e > hi || e < lo) v[e] = __float_as_uint(-INFINITY);
+              for (int k = 0; k < 32; ++k)
+                v[32 * q + k] = ((keep >> k) & 1u) ? v[32 * q + k] : __float_as_uint(-INFINITY);
             }
           }
         }
