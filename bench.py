@@ -103,9 +103,9 @@ def decode_mq_bytes(c, lens) -> int:
 # hash to the recorded digest, else null.
 PREFILL_TRAFFIC = {
     # prefill.cuh and ptx.cuh as captured; any change makes the figures stale
-    "source_sha256": "8197f1fa94111682cb2ae8c05745fe13fd349c63a67b9376b8c219b88d7a3aec",
-    "bytes": {"step37_sliding_B1_S8192_Hq96_Hkv8_W512": 394.6e6,
-              "step37_full_B1_S32768_Hq64_Hkv8_causal": 3997.6e6},
+    "source_sha256": "df9149fc28d156185721535bdda270f7e6de674db1f18509951db38bc88b8ae5",
+    "bytes": {"step37_sliding_B1_S8192_Hq96_Hkv8_W512": 399.2e6,
+              "step37_full_B1_S32768_Hq64_Hkv8_causal": 4076.7e6},
 }
 PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh")
 
