@@ -333,36 +333,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^y for a pair of floats on the FMA pipe instead of the SFU (which the
-// softmax otherwise saturates).  y is clamped to >= -127 and split as
-// y = n + f, n = round(y) via the 1.5 * 2^23 rounding constant, f in
-// [-1/2, 1/2]; 2^f comes from a cubic with constant term exactly 1 (minimax
-// relative error 1.01e-4 on the interval, fitted by tests/exp2_poly_fit.py)
-// and n is added into the exponent field.  Inputs at or below
-// -127, -inf included, give +0.0 exactly: n = -127, f = 0, and the sum of the
-// bit patterns of 1.0 and -127 << 23 wraps to zero.  For y in [-126, 127] the
-// result is within that relative error of 2^y; between -127 and -126 it is a
-// non-negative value below 2^-126 (no implicit leading one in a zero exponent
-// field), which a softmax row sum of at least 1 cannot see.  NaN inputs are
-// not handled.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t y) {
-  float y0, y1;
-  f2_unpack(y, y0, y1);
-  const uint64_t yc = f2_pack(fmaxf(y0, -127.f), fmaxf(y1, -127.f));
-  const uint64_t kRound = f2_pack(12582912.f, 12582912.f);
-  const uint64_t t = f2_add(yc, kRound);
-  const uint64_t r = f2_add(t, f2_pack(-12582912.f, -12582912.f));
-  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), yc);
-  uint64_t q = f2_fma(f2_pack(5.500892922e-02f, 5.500892922e-02f), f, f2_pack(2.422109544e-01f, 2.422109544e-01f));
-  q = f2_fma(q, f, f2_pack(6.932829022e-01f, 6.932829022e-01f));
-  q = f2_fma(q, f, f2_pack(1.f, 1.f));
-  float t0, t1, q0, q1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(q, q0, q1);
-  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
-}
-
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialization may be scheduled while the kernel before it on the stream is
 // still running; grid_dependency_wait() returns once that kernel has
