@@ -126,6 +126,10 @@ def measured_prefill_traffic(workload: str):
     return None
 
 
+# idle before each extra prefill leg of the default run (seconds)
+LEG_IDLE_S = 2.0
+
+
 # B200 spec sheet (dense, no sparsity) figures, reported beside the measured
 # peaks: bf16 tensor 2.25 PFLOP/s; HBM3e 7.7 TB/s (HGX board figure)
 SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 7700.0}
@@ -649,31 +653,38 @@ def main():
         # the extra legs and the CPU baseline describe one GPU: single-process runs only
         if world == 1 and args.only == "all":
             # the other prefill workloads, each timed like the headline
-            # (rotating input sets, CUDA events around the steps)
+            # (rotating input sets, CUDA events around the steps, clocks
+            # sampled).  Each starts after LEG_IDLE_S of idle: right after
+            # the headline's kilowatt steps the power controller still holds
+            # the SM clock down, and a short leg would be timed in that tail.
             legs = {}
             for pc in (configs.STEP_SLIDING, configs.STEP_FULL, configs.MUSE_SLIDING, configs.MUSE_FULL):
                 if pc.name == c.name:
-                    p_ms, p_steps = ms, args.steps
+                    p_ms, p_steps, p_clk = ms, args.steps, clocks
                 else:
                     p_steps = max(5, min(200, int(200.0 / max(prefill_flops(pc) / 1e12, 1e-3))))
-                    p_ms, _, _ = bench_prefill(pc, p_steps, 3, dev, n_rotate=max(args.rotate, 1), clocks_on=False)
+                    time.sleep(LEG_IDLE_S)
+                    p_ms, p_clk, _ = bench_prefill(pc, p_steps, 3, dev, n_rotate=max(args.rotate, 1))
                 tf = prefill_flops(pc) / (p_ms / p_steps / 1e3) / 1e12
                 legs[pc.name] = {"ms": p_ms / p_steps, "steps": p_steps, "TFLOP/s": tf,
                                  "frac_bf16": tf / peaks["bf16_tflops"], "frac_of_spec": tf / SPEC_PEAKS["bf16_tflops"],
                                  "peak_source": f"{peak_src} bf16 burst", "unmasked_flop": prefill_flops(pc),
-                                 "traffic": measured_prefill_traffic(pc.name),
-                                 "timing": "swa_attn_prefill (key pre-pass + attention), CUDA events"}
+                                 "traffic": measured_prefill_traffic(pc.name), "clocks": p_clk,
+                                 "timing": "swa_attn_prefill (key pre-pass + attention), CUDA events"
+                                           + ("" if pc.name == c.name else f", after {LEG_IDLE_S:g} s idle")}
             line["prefill"] = legs
             assert api.device_error() == 0, "a kernel reported a bounded-wait timeout"
         if world == 1 and not args.no_decode and args.only == "all":
             # the short legs first, the two 34 GB full-layer decode legs last
             chunks = {}
             for cc in (configs.CHUNK_SLIDING, configs.CHUNK_FULL):
+                time.sleep(LEG_IDLE_S)
                 c_ms = bench_prefill_chunk(cc, 20 if cc.window > 0 else 5, 3, dev)
                 tf = chunk_flops(cc) / (c_ms / 1e3) / 1e12
                 chunks[cc.name] = {"ms": c_ms, "TFLOP/s": tf, "frac_bf16": tf / peaks["bf16_tflops"],
                                    "frac_of_spec": tf / SPEC_PEAKS["bf16_tflops"],
-                                   "peak_source": f"{peak_src} bf16 burst"}
+                                   "peak_source": f"{peak_src} bf16 burst",
+                                   "timing": f"CUDA events, after {LEG_IDLE_S:g} s idle"}
             extra, mqs = {}, {}
             for kind, dc in (("decode", configs.DECODE_SLIDING), ("mq", configs.MQ_SLIDING),
                              ("decode", configs.DECODE_FULL), ("mq", configs.MQ_FULL)):
