@@ -106,7 +106,9 @@ PREFILL_TRAFFIC = {
     # prefill kernel never called); any change makes the figures stale
     "source_sha256": "5651776bb5640ad70a5762b096e8397bef9f72a04bee8e7c60997f9efb642e55",
     "bytes": {"step37_sliding_B1_S8192_Hq96_Hkv8_W512": 399.2e6,
-              "step37_full_B1_S32768_Hq64_Hkv8_causal": 4076.7e6},
+              "step37_full_B1_S32768_Hq64_Hkv8_causal": 4076.7e6,
+              "muse_sliding_B4_S16384_Hq32_Hkv2_W2048": 1116.6e6,
+              "muse_full_B4_S16384_Hq32_Hkv2_causal_norope": 1784.2e6},
 }
 PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh")
 
