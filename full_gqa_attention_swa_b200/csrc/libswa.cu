@@ -267,8 +267,7 @@ std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_decode_scratch on the current device, looked up once
-// per device (the first call on a device does this; it must not run under
-// stream capture).
+// per device (the first call on a device does this).
 swa_status scratch_for_current_device(void** ptr) {
   int dev = 0;
   swa_status st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");

@@ -325,10 +325,10 @@ SWA_API const char* swa_version(void);
  * or different host threads, without ordering between them) race on it and
  * may return wrong results.  Order such calls on one stream or with events.
  *
- * The first call on each device does a one-time set-up (it looks up the
+ * The first call on each device does a one-time set-up: it looks up the
  * device address of the array with cudaGetSymbolAddress while that device is
- * current); make that first call before any stream capture.  The call itself
- * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * current.  The call itself allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.
  */
 #define SWA_NO_ALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
