@@ -62,8 +62,8 @@ constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
 // setmaxnreg split of the 128 x 512 registers the CTA is launched with
 constexpr uint32_t kRegsLaunch = 128;
-constexpr uint32_t kRegsSoftmax = 176;
-constexpr uint32_t kRegsCorrection = 104;
+constexpr uint32_t kRegsSoftmax = 184;
+constexpr uint32_t kRegsCorrection = 88;
 constexpr uint32_t kRegsOther = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCorrection + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");

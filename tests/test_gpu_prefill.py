@@ -43,6 +43,18 @@ def test_window_sweep(cuda_device, W, Hq):
     check_no_device_error()
 
 
+@pytest.mark.parametrize("W", [128, 256, 384, 512])
+def test_band_edge_on_tile_boundary(cuda_device, W):
+    """W a multiple of 128: for query tiles at or past position W the band's
+    first key tile is visible exactly above each row's diagonal and the
+    diagonal key tile exactly on and below it, the two masks complementary.
+    Every row is checked, with a ragged last tile and two head pairs per
+    kv-head."""
+    p = api.LayerParams(8, 2, 128, W, 1e4, 128)
+    _check_all_rows(cuda_device, p, 1, 1100, seed=900 + W)
+    check_no_device_error()
+
+
 @pytest.mark.parametrize("S", [1, 17, 128, 129, 255, 257, 640])
 @pytest.mark.parametrize("W", [64, -1])
 def test_ragged_lengths(cuda_device, S, W):

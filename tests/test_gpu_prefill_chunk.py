@@ -64,6 +64,15 @@ def test_sliding_chunks(cuda_device, bounds, W):
     _check(cuda_device, p, 2, bounds, seed=900 + W, C=W)
 
 
+@pytest.mark.parametrize("W,bounds", [(256, [0, 128, 640]), (512, [0, 384, 1000]), (384, [0, 256, 900])])
+def test_sliding_chunks_tile_aligned_history(cuda_device, W, bounds):
+    """A chunk whose history (the earlier tokens it attends to) is a multiple
+    of 128 long puts its query tiles on key tile boundaries: for W a multiple
+    of 128 the band's edges then fall exactly on key tile edges."""
+    p = api.LayerParams(8, 2, 128, W, 1e4, 128)
+    _check(cuda_device, p, 2, bounds, seed=950 + W, C=W)
+
+
 @pytest.mark.parametrize("bounds", [[0, 300], [0, 100, 137, 400], [0, 1, 2, 130, 131, 390], [0, 256, 640]],
                          ids=["one", "odd", "tiny-steps", "aligned"])
 @pytest.mark.parametrize("theta,r", [(5e6, 64), (0.0, 128)])
