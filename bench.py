@@ -102,13 +102,12 @@ def decode_mq_bytes(c, lens) -> int:
 # taken on, so it is reported only while csrc/prefill.cuh and csrc/ptx.cuh still
 # hash to the recorded digest, else null.
 PREFILL_TRAFFIC = {
-    # prefill.cuh and ptx.cuh as captured (ptx.cuh since lost one function the
-    # prefill kernel never called); any change makes the figures stale
-    "source_sha256": "5651776bb5640ad70a5762b096e8397bef9f72a04bee8e7c60997f9efb642e55",
-    "bytes": {"step37_sliding_B1_S8192_Hq96_Hkv8_W512": 399.2e6,
-              "step37_full_B1_S32768_Hq64_Hkv8_causal": 4076.7e6,
-              "muse_sliding_B4_S16384_Hq32_Hkv2_W2048": 1116.6e6,
-              "muse_full_B4_S16384_Hq32_Hkv2_causal_norope": 1784.2e6},
+    # prefill.cuh and ptx.cuh as captured; any change makes the figures stale
+    "source_sha256": "0655f30c06d1c348b18a77fad0b06b7992028d6865f28fc5a29449d239a48043",
+    "bytes": {"step37_sliding_B1_S8192_Hq96_Hkv8_W512": 399.4e6,
+              "step37_full_B1_S32768_Hq64_Hkv8_causal": 4368.3e6,
+              "muse_sliding_B4_S16384_Hq32_Hkv2_W2048": 1116.2e6,
+              "muse_full_B4_S16384_Hq32_Hkv2_causal_norope": 1754.3e6},
 }
 PREFILL_SOURCES = ("prefill.cuh", "ptx.cuh")
 
