@@ -60,6 +60,26 @@ def test_sliding_ring(cuda_device, W, G, T):
     check_no_device_error()
 
 
+@pytest.mark.parametrize("B,Hkv,G,W,T", [(1, 2, 8, 2048, 4), (2, 2, 8, 2048, 4), (39, 3, 4, 64, 3),
+                                         (64, 1, 12, 512, 4)],
+                         ids=["long-ring-splits", "long-and-short-ring", "many-rings", "full-rings"])
+def test_ring_batches(cuda_device, B, Hkv, G, W, T):
+    """Ring layers at other batch shapes: a long ring split over several CTAs
+    (merged from their partials), a long and a short ring in one batch, many
+    short rings, and a batch of full rings."""
+    p = api.LayerParams(G * Hkv, Hkv, 128, W, 1e4, 128)
+    rng = np.random.default_rng(2150 + B)
+    if B == 1:
+        lens = [T + 5000]
+    elif B == 2:
+        lens = [T + 5000, T + 100]
+    else:
+        lens = [int(x) for x in rng.integers(T, T + 5 * W, B)]
+    out, ref = _run(cuda_device, p, B, T, W, lens, seed=2160 + B + W)
+    assert_close(out, ref, f"mq ring batch B{B} Hkv{Hkv} G{G} W{W} T{T}")
+    check_no_device_error()
+
+
 @pytest.mark.parametrize("T", [1, 3, 4])
 @pytest.mark.parametrize("G", [2, 8, 16])
 def test_full_linear(cuda_device, G, T):
